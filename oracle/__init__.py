@@ -1,0 +1,246 @@
+"""CPU oracle for the FP8 runtime linear path -- TEST INFRASTRUCTURE ONLY.
+
+Only the test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library
+(``fp8_dynamic_scaled_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``fp8_oracle.c`` (plain C, IEEE binary32 without
+contraction for the fp32 steps, fp64 for the GEMM reference); this module only
+builds it with gcc and marshals numpy arrays through ctypes.  The independent
+NumPy nearest-code encoder in ``numpy_encoder.py`` is a second opinion used by
+the pin tests.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+E4M3, E5M2 = 0, 1
+TENSOR, ROW, BLOCK_1x128, BLOCK_128x128, MX32, DELAYED = 0, 1, 2, 3, 4, 5
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile fp8_oracle.c into liboracle.so with gcc (no fast-math, no FMA contraction)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+           "-shared", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    P, I64, I32, D, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_float
+    lib.orc_fmax.restype, lib.orc_fmax.argtypes = D, [I32]
+    lib.orc_decode.restype, lib.orc_decode.argtypes = D, [ctypes.c_uint8, I32]
+    lib.orc_encode.restype, lib.orc_encode.argtypes = ctypes.c_uint8, [D, I32]
+    lib.orc_encode_bruteforce.restype = ctypes.c_uint8
+    lib.orc_encode_bruteforce.argtypes = [D, I32]
+    lib.orc_scale_from_amax.restype, lib.orc_scale_from_amax.argtypes = F, [F, I32]
+    lib.orc_mx_exponent.restype, lib.orc_mx_exponent.argtypes = I32, [F]
+    lib.orc_f32_to_bf16.restype, lib.orc_f32_to_bf16.argtypes = ctypes.c_uint16, [F]
+    lib.orc_scale_count.restype, lib.orc_scale_count.argtypes = I64, [I32, I64, I64]
+    lib.orc_quantize.restype = I32
+    lib.orc_quantize.argtypes = [P, I64, I64, I64, I32, I32, P, P, P]
+    lib.orc_delayed_step.restype = I32
+    lib.orc_delayed_step.argtypes = [P, I64, I64, I64, I32, P, ctypes.c_int32, I64, P, P, P, P]
+    lib.orc_gemm_ref_points.restype = I32
+    lib.orc_gemm_ref_points.argtypes = [P, P, I32, I32, P, P, I32, I32, I64, I64, I64,
+                                        P, P, I64, P, P]
+    lib.orc_gemm_ref_full.restype = I32
+    lib.orc_gemm_ref_full.argtypes = [P, P, I32, I32, P, P, I32, I32, I64, I64, I64, P, P]
+    lib.orc_decode_table.restype, lib.orc_decode_table.argtypes = None, [I32, P]
+    for name in ("orc_encode_array", "orc_encode_bruteforce_array"):
+        getattr(lib, name).restype = None
+        getattr(lib, name).argtypes = [P, I64, I32, P]
+    lib.orc_f32_to_bf16_array.restype, lib.orc_f32_to_bf16_array.argtypes = None, [P, I64, P]
+    lib.orc_quant_scaled_array.restype = None
+    lib.orc_quant_scaled_array.argtypes = [P, I64, F, I32, P]
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def fmax(fmt: int) -> float:
+    return _load().orc_fmax(fmt)
+
+
+def decode(code: int, fmt: int) -> float:
+    return _load().orc_decode(code, fmt)
+
+
+def decode_table(fmt: int) -> np.ndarray:
+    out = np.empty(256, np.float64)
+    _load().orc_decode_table(fmt, _ptr(out))
+    return out
+
+
+def encode(values, fmt: int) -> np.ndarray:
+    v = np.ascontiguousarray(values, dtype=np.float32).ravel()
+    out = np.empty(v.size, np.uint8)
+    _load().orc_encode_array(_ptr(v), v.size, fmt, _ptr(out))
+    return out
+
+
+def encode_bruteforce(values, fmt: int) -> np.ndarray:
+    v = np.ascontiguousarray(values, dtype=np.float32).ravel()
+    out = np.empty(v.size, np.uint8)
+    _load().orc_encode_bruteforce_array(_ptr(v), v.size, fmt, _ptr(out))
+    return out
+
+
+def quant_scaled(values, s: float, fmt: int) -> np.ndarray:
+    """Codes of fp32 values under one fp32 scale: encode(clip(fp32(x / s)))."""
+    v = np.ascontiguousarray(values, dtype=np.float32).ravel()
+    out = np.empty(v.size, np.uint8)
+    _load().orc_quant_scaled_array(_ptr(v), v.size, float(s), fmt, _ptr(out))
+    return out
+
+
+def f32_to_bf16(values) -> np.ndarray:
+    v = np.ascontiguousarray(values, dtype=np.float32).ravel()
+    out = np.empty(v.size, np.uint16)
+    _load().orc_f32_to_bf16_array(_ptr(v), v.size, _ptr(out))
+    return out.reshape(np.shape(values))
+
+
+def scale_from_amax(amax: float, fmt: int) -> float:
+    return _load().orc_scale_from_amax(amax, fmt)
+
+
+def mx_exponent(amax: float) -> int:
+    return _load().orc_mx_exponent(amax)
+
+
+def scale_shape(mode: int, rows: int, cols: int):
+    if mode in (TENSOR, DELAYED):
+        return (1,)
+    if mode == ROW:
+        return (rows,)
+    if mode == BLOCK_1x128:
+        return (rows, -(-cols // 128))
+    if mode == BLOCK_128x128:
+        return (-(-rows // 128), -(-cols // 128))
+    if mode == MX32:
+        return (rows, cols // 32)
+    raise ValueError(mode)
+
+
+def quantize(x_bf16: np.ndarray, fmt: int, mode: int, dequant: bool = True):
+    """Quantize a bf16 matrix (uint16 bit patterns, [rows, cols] or a strided view).
+
+    Returns (codes uint8 [rows, cols], scale (float32, or uint8 E8M0 for MX32),
+    dequant uint16 bf16 bits [rows, cols] or None).
+    """
+    assert x_bf16.dtype == np.uint16 and x_bf16.ndim == 2
+    rows, cols = x_bf16.shape
+    if x_bf16.strides[1] != 2 or x_bf16.strides[0] % 2 or x_bf16.strides[0] < 2 * cols:
+        x_bf16 = np.ascontiguousarray(x_bf16)
+    ld = x_bf16.strides[0] // 2 if rows > 0 else cols
+    ptr = x_bf16.ctypes.data      # row-strided view: rows start ld elements apart
+    q = np.empty((rows, cols), np.uint8)
+    sdt = np.uint8 if mode == MX32 else np.float32
+    scale = np.empty(scale_shape(mode, rows, cols), sdt)
+    deq = np.empty((rows, cols), np.uint16) if dequant else None
+    rc = _load().orc_quantize(ptr, rows, cols, ld, fmt, mode, _ptr(q), _ptr(scale), _ptr(deq))
+    if rc != 0:
+        raise OracleError(f"orc_quantize failed: {rc} ({'non-finite input' if rc == 1 else 'bad argument'})")
+    return q, scale, deq
+
+
+def delayed_step(x_bf16: np.ndarray, fmt: int, ring: np.ndarray, t: int, dequant: bool = False):
+    """One delayed-scaling step; updates ``ring`` (float32[h]) in place.
+
+    Returns (codes, scale float32, dequant or None, saturated element count).
+    """
+    assert x_bf16.dtype == np.uint16 and x_bf16.ndim == 2 and x_bf16.flags["C_CONTIGUOUS"]
+    assert ring.dtype == np.float32 and ring.flags["C_CONTIGUOUS"]
+    rows, cols = x_bf16.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty(1, np.float32)
+    sat = np.zeros(1, np.int64)
+    deq = np.empty((rows, cols), np.uint16) if dequant else None
+    rc = _load().orc_delayed_step(_ptr(x_bf16), rows, cols, cols, fmt, _ptr(ring), ring.size, t,
+                                  _ptr(q), _ptr(s), _ptr(deq), _ptr(sat))
+    if rc != 0:
+        raise OracleError(f"orc_delayed_step failed: {rc}")
+    return q, s[0], deq, int(sat[0])
+
+
+def gemm_ref_full(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b):
+    """fp64 reference Y = A_deq B_deq^T and bound sum_k |terms|; a [M,K], b [N,K] codes."""
+    M, K = a.shape
+    N = b.shape[0]
+    y = np.empty((M, N), np.float64)
+    bound = np.empty((M, N), np.float64)
+    rc = _load().orc_gemm_ref_full(_ptr(np.ascontiguousarray(a)), _ptr(np.ascontiguousarray(sa)),
+                                   a_mode, fmt_a, _ptr(np.ascontiguousarray(b)),
+                                   _ptr(np.ascontiguousarray(sb)), b_mode, fmt_b, M, N, K,
+                                   _ptr(y), _ptr(bound))
+    if rc != 0:
+        raise OracleError("orc_gemm_ref_full failed")
+    return y, bound
+
+
+def gemm_ref_points(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b, pm, pn):
+    """fp64 reference at output points (pm[i], pn[i]); returns (y, bound)."""
+    M, K = a.shape
+    N = b.shape[0]
+    pm = np.ascontiguousarray(pm, dtype=np.int64)
+    pn = np.ascontiguousarray(pn, dtype=np.int64)
+    order = np.argsort(pm, kind="stable")
+    y = np.empty(pm.size, np.float64)
+    bound = np.empty(pm.size, np.float64)
+    pm_s, pn_s = np.ascontiguousarray(pm[order]), np.ascontiguousarray(pn[order])
+    ys = np.empty_like(y)
+    bs = np.empty_like(bound)
+    rc = _load().orc_gemm_ref_points(_ptr(np.ascontiguousarray(a)), _ptr(np.ascontiguousarray(sa)),
+                                     a_mode, fmt_a, _ptr(np.ascontiguousarray(b)),
+                                     _ptr(np.ascontiguousarray(sb)), b_mode, fmt_b, M, N, K,
+                                     _ptr(pm_s), _ptr(pn_s), pm.size, _ptr(ys), _ptr(bs))
+    if rc != 0:
+        raise OracleError("orc_gemm_ref_points failed")
+    y[order] = ys
+    bound[order] = bs
+    return y, bound
+
+
+def bf16_ulp(y: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |y| (8 significant bits; subnormal floor 2^-133)."""
+    a = np.abs(np.asarray(y, np.float64))
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -126.0)
+    return np.where(a > 0, np.exp2(e - 7.0), 2.0 ** -133)
+
+
+def gemm_within_tolerance(y_gpu, y_ref, bound, rel: float = 1e-3):
+    """The GEMM acceptance rule: |y - y_ref| <= rel * sum_k|terms| + 1 bf16 ulp of y_ref."""
+    err = np.abs(np.asarray(y_gpu, np.float64) - y_ref)
+    lim = rel * bound + bf16_ulp(y_ref)
+    return err <= lim, err, lim
