@@ -1,0 +1,578 @@
+// gemm_sm100.cu -- FP8 scaled GEMM on the 5th-generation tensor cores (sm_100a).
+//
+//   Y[m, n] = bf16( sum_k S_a(m,k) a[m,k] * S_b(n,k) b[n,k] ),  A [M,K], B [N,K] K-major
+//
+// [FFS] "FP8 formats, scaling and LLM inference", section "一次 FP8 GEMM 的完整精度契约":
+// Y ~= s_x s_w (X_8 W_8) with the products accumulated in higher precision and a
+// BF16 output; [PQG] "FP8 产线量化落地指南", code fp8_gemm_forward (out_dtype bf16).
+//
+// Structure (one persistent CTA per SM, warp-specialised):
+//   warp 0       TMA producer: 128-byte-swizzled A/B tiles into a STAGES-deep ring
+//   warp 1       TMEM allocator + MMA issuer: tcgen05.mma kind::f8f6f4 (or
+//                kind::mxf8f6f4.block_scale), M=128 N=256 K=32 per instruction,
+//                FP32 accumulators in TMEM, tcgen05.commit -> mbarriers
+//   warp 2       (MX only) scale-factor warp: E8M0 bytes into the layout tcgen05.cp wants
+//   epilogue     4 warps (ROWSCALE) or 8 warps (BLOCK, MX): tcgen05.ld -> scale ->
+//                bf16 -> swizzled smem -> TMA store
+// Variants:
+//   ROWSCALE  per-tensor / per-row scales applied in the epilogue; accumulators
+//             double-buffered in TMEM (2 x 256 columns) so the epilogue of tile i
+//             overlaps the mainloop of tile i+1.
+//   BLOCK     1x128 activation blocks x 128x128 weight blocks: every 128-deep K block
+//             is accumulated into its own TMEM buffer; the epilogue promotes it into
+//             FP32 registers with s_x[m,kb] * s_w[n/128,kb] (software promotion).
+//   MX        MXFP8: E8M0 scales for every 32 K of each row/column are copied into
+//             TMEM and applied by the tensor core itself.
+// Every mbarrier wait is bounded (globaltimer); on expiry the CTA raises an abort
+// flag, reports FP8_ERR_TIMEOUT in dev_status, drains and frees TMEM, and exits.
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace fp8b {
+
+constexpr int BM = 128;             // rows of A per tile (TMEM lanes)
+constexpr int BN = 256;             // rows of B per tile (TMEM columns)
+constexpr int BK = 128;             // K bytes per pipeline stage (one 128-byte swizzle row)
+constexpr int UMMA_K = 32;          // K per tcgen05.mma for 8-bit operands
+constexpr int STAGES = 4;
+constexpr uint32_t A_STAGE_BYTES = BM * BK;   // 16 KB
+constexpr uint32_t B_STAGE_BYTES = BN * BK;   // 32 KB
+constexpr uint64_t WAIT_TIMEOUT_NS = 4000000000ull;   // 4 s
+
+enum Variant { V_ROWSCALE = 0, V_BLOCK = 1, V_MX = 2 };
+
+template <int V> struct Cfg;
+template <> struct Cfg<V_ROWSCALE> {
+    static constexpr int EPI_WARPS = 4, FIRST_EPI_WARP = 2, STAGE_BUFS = 2;
+    static constexpr int ACC_BUFS = 2;            // TMEM accumulators of BN columns
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+template <> struct Cfg<V_BLOCK> {
+    static constexpr int EPI_WARPS = 8, FIRST_EPI_WARP = 2, STAGE_BUFS = 2;
+    static constexpr int ACC_BUFS = 2;            // per-K-block partial products
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+template <> struct Cfg<V_MX> {
+    static constexpr int EPI_WARPS = 8, FIRST_EPI_WARP = 3, STAGE_BUFS = 1;
+    static constexpr int ACC_BUFS = 1;            // + scale factors in columns 256..267
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+constexpr uint32_t SF_STAGE_BYTES = 512 * 3;  // MX: 128 A rows + 256 B rows, 4 bytes each
+
+template <int V>
+struct Smem {
+    static constexpr int NT = 32 * (Cfg<V>::FIRST_EPI_WARP + Cfg<V>::EPI_WARPS);
+    static constexpr uint32_t A_OFF = 0;
+    static constexpr uint32_t B_OFF = A_OFF + STAGES * A_STAGE_BYTES;
+    static constexpr uint32_t Y_OFF = B_OFF + STAGES * B_STAGE_BYTES;
+    static constexpr uint32_t Y_BYTES = Cfg<V>::EPI_WARPS * Cfg<V>::STAGE_BUFS * 2048;
+    static constexpr uint32_t SF_OFF = Y_OFF + Y_BYTES;
+    static constexpr uint32_t SF_BYTES = V == V_MX ? STAGES * SF_STAGE_BYTES : 0;
+    static constexpr uint32_t BAR_OFF = SF_OFF + SF_BYTES;
+    // full[S], empty[S], tfull[2], tempty[2], teardown
+    static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 4 + 1);
+    static constexpr uint32_t MISC_OFF = BAR_OFF + BAR_BYTES;   // tmem slot, abort flag
+    static constexpr uint32_t TOTAL = MISC_OFF + 16;
+    static constexpr uint32_t ALLOC = TOTAL + 1024;             // slack for 1024-B alignment
+};
+
+struct GemmParams {
+    int32_t M, N, K;
+    int32_t num_m, num_n, num_kb;
+    int32_t m_fastest;
+    // ROWSCALE: element scale = sa[m * sa_stride] * sb[n * sb_stride]
+    const float* sa;
+    const float* sb;
+    int32_t sa_stride, sb_stride;
+    // BLOCK: sa [M][num_kb], sb [ceil(N/128)][num_kb];  MX: E8M0 bytes [rows][K/32]
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    uint32_t idesc;
+    int32_t* status;
+};
+
+// ---------------------------------------------------------------- bounded waits
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
+                                             int32_t* status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+            *abort_flag = 1;
+            report_status(status, FP8_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int32_t t, int32_t& mb, int32_t& nb) {
+    if (p.m_fastest) { mb = t % p.num_m; nb = t / p.num_m; }
+    else             { nb = t % p.num_n; mb = t / p.num_n; }
+}
+
+// Write 32 bf16 (16 packed words) of one row into a 32x32 staging tile laid out
+// for the 64-byte TMA swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r>>1)&3).
+__device__ __forceinline__ void stage_row_sw64(uint8_t* buf, int r, const uint32_t (&w)[16]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int jj = j ^ ((r >> 1) & 3);
+        *reinterpret_cast<uint4*>(buf + r * 64 + jj * 16) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    }
+}
+
+// Store a 32-row x 32-column bf16 chunk held one row per lane.
+__device__ __forceinline__ void store_chunk(const CUtensorMap* tmY, uint8_t* buf, const uint32_t (&w)[16],
+                                            int32_t x, int32_t y, int lane) {
+    stage_row_sw64(buf, lane, w);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        ptx::tma_store_2d(tmY, buf, x, y);
+        ptx::bulk_commit();
+    }
+}
+
+// ================================================================ the kernel
+template <int V>
+__global__ void __launch_bounds__(Smem<V>::NT, 1)
+fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+    using C = Cfg<V>;
+    using S = Smem<V>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem + S::A_OFF;
+    uint8_t* sB = smem + S::B_OFF;
+    uint8_t* sY = smem + S::Y_OFF;
+    uint8_t* sSF = smem + S::SF_OFF;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* teardown = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::MISC_OFF);
+    volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + S::MISC_OFF + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int32_t num_tiles = p.num_m * p.num_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&full[s], V == V_MX ? 2 : 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], C::EPI_WARPS);
+        }
+        ptx::mbar_init(teardown, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        ptx::prefetch_tmap(&tmY);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                int32_t mb, nb;
+                tile_coords(p, t, mb, nb);
+                for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&full[stage], A_STAGE_BYTES + B_STAGE_BYTES);
+                    ptx::tma_load_2d(sA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, mb * BM);
+                    ptx::tma_load_2d(sB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        uint32_t stage = 0, phase = 0;
+        uint32_t acc_it = 0;       // accumulator-buffer use counter
+        bool ok = true;
+        const uint32_t sA0 = ptx::smem_u32(sA), sB0 = ptx::smem_u32(sB), sSF0 = ptx::smem_u32(sSF);
+        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            if (V != V_BLOCK) {
+                const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
+                if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+            }
+            for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                if (V == V_BLOCK) {
+                    const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
+                    if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                }
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (acc_it % C::ACC_BUFS) * BN;
+                if (lane == 0) {
+                    if (V == V_MX) {
+                        const uint32_t sf = sSF0 + stage * SF_STAGE_BYTES;
+                        ptx::tmem_cp_32x128b_x4(tmem_base + 256, ptx::sdesc_plain_128b(sf));
+                        ptx::tmem_cp_32x128b_x4(tmem_base + 260, ptx::sdesc_plain_128b(sf + 512));
+                        ptx::tmem_cp_32x128b_x4(tmem_base + 264, ptx::sdesc_plain_128b(sf + 1024));
+                    }
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        const uint64_t ad = ptx::sdesc_kmajor_sw128(sA0 + stage * A_STAGE_BYTES + k * UMMA_K);
+                        const uint64_t bd = ptx::sdesc_kmajor_sw128(sB0 + stage * B_STAGE_BYTES + k * UMMA_K);
+                        if (V == V_MX) {
+                            // A and B scale-factor ids select byte k of each TMEM word
+                            const uint32_t id = p.idesc | ((uint32_t)k << 29) | ((uint32_t)k << 4);
+                            ptx::mma_mxf8f6f4(d_tmem, ad, bd, id, tmem_base + 256, tmem_base + 260,
+                                              (kb | k) != 0);
+                        } else if (V == V_BLOCK) {
+                            ptx::mma_f8f6f4(d_tmem, ad, bd, p.idesc, k != 0);
+                        } else {
+                            ptx::mma_f8f6f4(d_tmem, ad, bd, p.idesc, (kb | k) != 0);
+                        }
+                    }
+                    ptx::mma_commit(&empty[stage]);
+                    if (V == V_BLOCK) ptx::mma_commit(&tfull[acc_it % C::ACC_BUFS]);
+                }
+                __syncwarp();
+                if (V == V_BLOCK) ++acc_it;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            if (V != V_BLOCK) {
+                if (lane == 0) ptx::mma_commit(&tfull[acc_it % C::ACC_BUFS]);
+                __syncwarp();
+                ++acc_it;
+            }
+        }
+        // all issued tcgen05 work must finish before TMEM is released
+        if (lane == 0) {
+            ptx::mma_commit(teardown);
+            wait_bounded(teardown, 0, abort_flag, p.status);
+        }
+        __syncwarp();
+    } else if (V == V_MX && warp == 2) {
+        // ------------------------------------------------ MX scale-factor warp
+        // Stage layout (what tcgen05.cp 32x128b.warpx4 reads): for a block of 128
+        // rows, byte (r % 32) * 16 + (r / 32) * 4 + j holds the scale of row r for
+        // the j-th 32-wide K slice of this 128-wide stage.
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        const int32_t kg = p.K / 32;                 // scale bytes per row
+        const bool aligned4 = (kg % 4) == 0 && ((reinterpret_cast<uintptr_t>(p.sfa) | reinterpret_cast<uintptr_t>(p.sfb)) & 3u) == 0;
+        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            int32_t mb, nb;
+            tile_coords(p, t, mb, nb);
+            for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                uint32_t w[12];
+#pragma unroll
+                for (int q = 0; q < 12; ++q) {
+                    const bool isA = q < 4;
+                    const int32_t row = isA ? mb * BM + lane + 32 * q : nb * BN + lane + 32 * (q - 4);
+                    const int32_t rows = isA ? p.M : p.N;
+                    const uint8_t* base = isA ? p.sfa : p.sfb;
+                    uint32_t v = 0x7F7F7F7Fu;      // 2^0 for rows past the edge (their codes are 0)
+                    if (row < rows) {
+                        const uint8_t* src = base + (int64_t)row * kg + kb * 4;
+                        if (aligned4 && kb * 4 + 4 <= kg) {
+                            v = __ldg(reinterpret_cast<const uint32_t*>(src));
+                        } else {
+                            v = 0;
+                            for (int j = 0; j < 4; ++j)
+                                v |= (uint32_t)(kb * 4 + j < kg ? __ldg(src + j) : 0x7Fu) << (8 * j);
+                        }
+                    }
+                    w[q] = v;
+                }
+                if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                uint8_t* dst = sSF + stage * SF_STAGE_BYTES;
+                *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(dst + 512 + lane * 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                *reinterpret_cast<uint4*>(dst + 1024 + lane * 16) = make_uint4(w[8], w[9], w[10], w[11]);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&full[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp >= C::FIRST_EPI_WARP) {
+        // ------------------------------------------------ epilogue
+        const int ew = warp - C::FIRST_EPI_WARP;          // 0 .. EPI_WARPS-1
+        const int quarter = warp & 3;                      // TMEM lane quarter this warp may access
+        const int half = (C::EPI_WARPS == 8) ? (ew >> 2) : 0;   // column half (8-warp variants)
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        uint8_t* ybuf = sY + ew * C::STAGE_BUFS * 2048;
+        uint32_t acc_it = 0;
+        uint32_t store_it = 0;
+        bool ok = true;
+        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            int32_t mb, nb;
+            tile_coords(p, t, mb, nb);
+            const int32_t row = mb * BM + quarter * 32 + lane;
+            const int32_t y_row0 = mb * BM + quarter * 32;
+            if (V == V_ROWSCALE) {
+                const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
+                if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const float sx = row < p.M ? __ldg(p.sa + (int64_t)row * p.sa_stride) : 0.0f;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_base + buf * BN + c * 32, r);
+                    ptx::tmem_ld_wait();
+                    if (c == BN / 32 - 1) {
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+                    }
+                    const int32_t n0 = nb * BN + c * 32;
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const int32_t n = n0 + j;
+                        const float s0 = n < p.N ? sx * __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
+                        const float s1 = n + 1 < p.N ? sx * __ldg(p.sb + (int64_t)(n + 1) * p.sb_stride) : 0.0f;
+                        w[j / 2] = pack_bf16x2(__uint_as_float(r[j]) * s0, __uint_as_float(r[j + 1]) * s1);
+                    }
+                    if (n0 < p.N) {
+                        uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
+                        if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
+                        __syncwarp();
+                        store_chunk(&tmY, b, w, n0, y_row0, lane);
+                        ++store_it;
+                    }
+                }
+                ++acc_it;
+            } else if (V == V_BLOCK) {
+                // software promotion over the K blocks
+                float acc[128];
+#pragma unroll
+                for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+                const int32_t nblk = nb * 2 + half;                      // 128-wide weight block
+                const int32_t nbw = (p.N + 127) / 128;
+                const float* sxr = p.sa + (int64_t)(row < p.M ? row : 0) * p.num_kb;
+                const float* swr = p.sb + (int64_t)(nblk < nbw ? nblk : 0) * p.num_kb;
+                float sx_next = __ldg(sxr), sw_next = __ldg(swr);
+                for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                    const float s = sx_next * sw_next;
+                    if (kb + 1 < p.num_kb) { sx_next = __ldg(sxr + kb + 1); sw_next = __ldg(swr + kb + 1); }
+                    const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
+                    if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) { ok = false; break; }
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[32];
+                        ptx::tmem_ld_32x32b_x32(tmem_base + lane_base + buf * BN + half * 128 + c * 32, r);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), s, acc[c * 32 + j]);
+                    }
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+                    ++acc_it;
+                }
+                if (!ok) break;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int32_t n0 = nb * BN + half * 128 + c * 32;
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) w[j / 2] = pack_bf16x2(acc[c * 32 + j], acc[c * 32 + j + 1]);
+                    if (n0 < p.N) {
+                        uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
+                        if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
+                        __syncwarp();
+                        store_chunk(&tmY, b, w, n0, y_row0, lane);
+                        ++store_it;
+                    }
+                }
+            } else {  // V_MX: drain the single accumulator into registers, then store
+                if (!wait_bounded(&tfull[0], acc_it & 1u, abort_flag, p.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                uint32_t r[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_base + half * 128 + c * 32, r[c]);
+                ptx::tmem_ld_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&tempty[0]);
+                ++acc_it;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int32_t n0 = nb * BN + half * 128 + c * 32;
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2)
+                        w[j / 2] = pack_bf16x2(__uint_as_float(r[c][j]), __uint_as_float(r[c][j + 1]));
+                    if (n0 < p.N) {
+                        uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
+                        if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
+                        __syncwarp();
+                        store_chunk(&tmY, b, w, n0, y_row0, lane);
+                        ++store_it;
+                    }
+                }
+            }
+        }
+        if (lane == 0) ptx::bulk_wait_all();
+        __syncwarp();
+    }
+
+    // ------------------------------------------------ teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ================================================================ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int V>
+static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaStream_t st) {
+    CUtensorMap ta, tb, ty;
+    // M, N, K sizes beyond 2^31 are rejected by the API before this point.
+    if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.K, BK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, (uint64_t)g.N, (uint64_t)g.M,
+                     (uint64_t)g.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)Smem<V>::ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    const int32_t tiles = p.num_m * p.num_n;
+    const int grid = std::max(1, std::min(tiles, num_sms()));
+    fp8_gemm_kernel<V><<<grid, Smem<V>::NT, Smem<V>::ALLOC, st>>>(ta, tb, ty, p);
+    return cudaGetLastError();
+}
+
+// Instruction descriptor, kind::f8f6f4: D = F32 (bits 4-5 = 1), A/B formats in bits
+// 7-9 / 10-12 (E4M3 = 0, E5M2 = 1), both K-major, N>>3 in bits 17-22, M>>4 in 24-28.
+static uint32_t idesc_f8f6f4(int fa, int fb) {
+    return (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+// kind::mxf8f6f4.block_scale: formats as above, scale format E8M0 (bit 23), the
+// scale-factor ids (bits 29-30 for A, 4-5 for B) are filled per instruction.
+static uint32_t idesc_mx(int fa, int fb) {
+    return ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
+    GemmParams p{};
+    p.M = (int32_t)g.M;
+    p.N = (int32_t)g.N;
+    p.K = (int32_t)g.K;
+    p.num_m = (int32_t)((g.M + BM - 1) / BM);
+    p.num_n = (int32_t)((g.N + BN - 1) / BN);
+    p.num_kb = (int32_t)((g.K + BK - 1) / BK);
+    // keep the operand with the smaller footprint resident in L2: walk its tiles fastest
+    p.m_fastest = (g.M <= g.N) ? 1 : 0;
+    p.status = g.status;
+    const bool a_pt = g.a_mode == FP8_SCALE_TENSOR || g.a_mode == FP8_SCALE_DELAYED;
+    const bool b_pt = g.b_mode == FP8_SCALE_TENSOR || g.b_mode == FP8_SCALE_DELAYED;
+    if ((a_pt || g.a_mode == FP8_SCALE_ROW) && (b_pt || g.b_mode == FP8_SCALE_ROW)) {
+        p.sa = static_cast<const float*>(g.sa);
+        p.sb = static_cast<const float*>(g.sb);
+        p.sa_stride = a_pt ? 0 : 1;
+        p.sb_stride = b_pt ? 0 : 1;
+        p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
+        return launch_variant<V_ROWSCALE>(g, p, st);
+    }
+    if (g.a_mode == FP8_SCALE_BLOCK_1x128 && g.b_mode == FP8_SCALE_BLOCK_128x128) {
+        p.sa = static_cast<const float*>(g.sa);
+        p.sb = static_cast<const float*>(g.sb);
+        p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
+        return launch_variant<V_BLOCK>(g, p, st);
+    }
+    if (g.a_mode == FP8_SCALE_MX32 && g.b_mode == FP8_SCALE_MX32) {
+        p.sfa = static_cast<const uint8_t*>(g.sa);
+        p.sfb = static_cast<const uint8_t*>(g.sb);
+        p.idesc = idesc_mx(g.fmt_a, g.fmt_b);
+        return launch_variant<V_MX>(g, p, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+__global__ void zero_rows_kernel(uint16_t* y, int64_t M, int64_t N, int64_t ldy) {
+    for (int64_t r = blockIdx.y; r < M; r += gridDim.y)
+        for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < N; c += (int64_t)gridDim.x * blockDim.x)
+            y[r * ldy + c] = 0;
+}
+
+cudaError_t launch_zero_output(uint16_t* y, int64_t M, int64_t N, int64_t ldy, cudaStream_t st) {
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    dim3 grid((unsigned)std::min<int64_t>((N + 255) / 256, 64), (unsigned)std::min<int64_t>(M, 1024));
+    zero_rows_kernel<<<grid, 256, 0, st>>>(y, M, N, ldy);
+    return cudaGetLastError();
+}
+
+}  // namespace fp8b

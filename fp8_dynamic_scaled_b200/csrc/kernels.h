@@ -1,0 +1,50 @@
+// kernels.h -- internal launcher interface between the C ABI (api.cu) and the
+// kernels (quantize.cu, gemm_sm100.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace fp8b {
+
+struct QuantArgs {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    int32_t fmt, mode;
+    uint8_t* q;
+    void* scale;
+    uint16_t* deq;          // nullable
+    int32_t* status;        // nullable
+    uint32_t* partials;     // per-tensor workspace (amax_partials_count() entries)
+    // delayed scaling (hist_ring == nullptr otherwise)
+    float* hist_ring;
+    int32_t hist_len;
+    int64_t hist_step;
+    float* hist_pending;
+    uint32_t* hist_ticket;
+};
+
+int32_t amax_partials_count();
+cudaError_t launch_quantize_tensor(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_quantize_grouped(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_fill_scale(float* s, int64_t n, float v, cudaStream_t st);
+
+struct GemmArgs {
+    const uint8_t* a;        // [M, K] codes
+    const uint8_t* b;        // [N, K] codes
+    const void* sa;
+    const void* sb;
+    int32_t a_mode, b_mode;  // TENSOR/ROW (any mix), BLOCK pair, or MX32 pair
+    int32_t fmt_a, fmt_b;
+    int64_t M, N, K;
+    uint16_t* y;             // bf16 [M, N], row stride ldy
+    int64_t ldy;
+    int32_t* status;
+};
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
+cudaError_t launch_zero_output(uint16_t* y, int64_t M, int64_t N, int64_t ldy, cudaStream_t st);
+
+}  // namespace fp8b

@@ -1,0 +1,523 @@
+// quantize.cu -- fused amax-reduce + scale + saturating RNE cast kernels (sm_100a).
+//
+// What is computed ([FFS] = "FP8 formats, scaling and LLM inference",
+// [PQG] = "FP8 产线量化落地指南"):
+//   a_max = max|x| over the scaling group          ([FFS] "Scale 怎样把 Tensor 塞进 E4M3", eq. a_max)
+//   s     = fp32(max(a_max, 1e-12f) / F_max)      ([FFS] eq. s = a_max/F_max; [PQG] code)
+//   q     = RNE_fp8(clip(fp32(x / s), +-F_max))   ([FFS] eq. X_fp8; [PQG] code step 3)
+//   d     = bf16_RNE(fp32(decode(q) * s))         ([FFS] eq. X^ = s X_fp8), optional
+// Groups: the whole tensor (TENSOR, DELAYED), a row (ROW), 1x128 and 128x128
+// blocks ([FFS] "Per-channel 与 Block Scaling", eq. s_g = a_g/F_max), and 32-element
+// MX blocks with a power-of-two scale 2^e, e = clamp(floor(log2 a_max) - 8, -127, 127).
+//
+// Data movement: every kernel reads bf16 with 16-byte vector loads that are
+// contiguous across a warp, and writes codes with 8-byte stores that are
+// contiguous across a warp.  amax is an integer max over the |bf16| bit
+// patterns (exact and order-free); a pattern >= 0x7F80 flags NaN/Inf input.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fp8b {
+
+constexpr int QT = 256;     // threads per CTA of the streaming kernels
+constexpr int VEC = 8;      // bf16 elements per 16-byte vector
+
+// ---------------------------------------------------------------- per-vector ops
+// |x| max over the 8 bf16 of a vector, as a packed pair of 16-bit patterns.
+__device__ __forceinline__ uint32_t vec_amax2(const uint4& v) {
+    uint32_t a = max_bf16x2_bits(abs_bf16x2(v.x), abs_bf16x2(v.y));
+    uint32_t b = max_bf16x2_bits(abs_bf16x2(v.z), abs_bf16x2(v.w));
+    return max_bf16x2_bits(a, b);
+}
+
+// How one element turns into the value that is cast: x / s (IEEE division) for
+// fp32 scales, x * 2^-e (exact) for MX scales.
+struct DivScale {
+    float s;
+    __device__ __forceinline__ float operator()(float x) const { return __fdiv_rn(x, s); }
+    __device__ __forceinline__ float deq() const { return s; }
+};
+struct Pow2Scale {
+    float inv;   // 2^-e
+    float mul;   // 2^e
+    __device__ __forceinline__ float operator()(float x) const { return __fmul_rn(x, inv); }
+    __device__ __forceinline__ float deq() const { return mul; }
+};
+
+// 8 elements -> 8 codes (byte i = element i).
+template <int FMT, class Op>
+__device__ __forceinline__ uint2 cast_vec(const uint4& v, const Op& op) {
+    uint32_t c0 = cvt_pair<FMT>(op(bf16_lo(v.x)), op(bf16_hi(v.x)));
+    uint32_t c1 = cvt_pair<FMT>(op(bf16_lo(v.y)), op(bf16_hi(v.y)));
+    uint32_t c2 = cvt_pair<FMT>(op(bf16_lo(v.z)), op(bf16_hi(v.z)));
+    uint32_t c3 = cvt_pair<FMT>(op(bf16_lo(v.w)), op(bf16_hi(v.w)));
+    return make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
+}
+
+// 8 codes -> 8 bf16 of decode(q) * mul.
+template <int FMT>
+__device__ __forceinline__ uint4 dequant_vec(const uint2& c, float mul) {
+    float2 a = decode_pair<FMT>(c.x & 0xFFFFu);
+    float2 b = decode_pair<FMT>(c.x >> 16);
+    float2 d = decode_pair<FMT>(c.y & 0xFFFFu);
+    float2 e = decode_pair<FMT>(c.y >> 16);
+    return make_uint4(pack_bf16x2(__fmul_rn(a.x, mul), __fmul_rn(a.y, mul)),
+                      pack_bf16x2(__fmul_rn(b.x, mul), __fmul_rn(b.y, mul)),
+                      pack_bf16x2(__fmul_rn(d.x, mul), __fmul_rn(d.y, mul)),
+                      pack_bf16x2(__fmul_rn(e.x, mul), __fmul_rn(e.y, mul)));
+}
+
+// MX shared exponent from an amax bf16 pattern: floor(log2 a) is the unbiased
+// exponent of a (bf16 subnormals: position of the leading mantissa bit).
+__device__ __forceinline__ int mx_exponent(uint32_t amax_bits) {
+    if (amax_bits == 0) return -127;
+    int ebits = (int)(amax_bits >> 7) & 0xFF;
+    int flog2;
+    if (ebits != 0) {
+        flog2 = ebits - 127;
+    } else {
+        int m = (int)(amax_bits & 0x7F);               // subnormal: m * 2^-133
+        flog2 = (31 - __clz(m)) - 133;
+    }
+    int e = flog2 - 8;
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^k as an fp32 value for k in [-149, 127] (exact).
+__device__ __forceinline__ float exp2i(int k) {
+    if (k >= -126) return __uint_as_float((uint32_t)(k + 127) << 23);
+    return __uint_as_float(1u << (k + 149));
+}
+
+// Block-wide max of a 32-bit pattern (all threads get the result).
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red /* [32] */) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    const int nw = blockDim.x >> 5;
+    uint32_t r = lane < nw ? red[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r = max(r, __shfl_xor_sync(0xffffffffu, r, o));
+    return r;
+}
+
+// ================================================================ per-tensor
+// Phase 1: each CTA writes the max |bf16| pattern over its share of the tensor.
+// The tensor is viewed as nrows rows of nvec 16-byte vectors (a dense tensor is
+// passed as one long row).
+__global__ void __launch_bounds__(QT) amax_partials_kernel(const uint16_t* __restrict__ x, int64_t nrows,
+                                                           int64_t nvec, int64_t ld,
+                                                           uint32_t* __restrict__ partials) {
+    __shared__ uint32_t red[32];
+    uint32_t m2 = 0;
+    const int64_t stride = (int64_t)gridDim.x * QT;
+    for (int64_t r = blockIdx.y; r < nrows; r += gridDim.y) {
+        const uint16_t* row = x + r * ld;
+        int64_t v = (int64_t)blockIdx.x * QT + threadIdx.x;
+        for (; v + 3 * stride < nvec; v += 4 * stride) {
+            uint4 a = ld_v4(row + v * VEC);
+            uint4 b = ld_v4(row + (v + stride) * VEC);
+            uint4 c = ld_v4(row + (v + 2 * stride) * VEC);
+            uint4 d = ld_v4(row + (v + 3 * stride) * VEC);
+            m2 = max_bf16x2_bits(m2, max_bf16x2_bits(max_bf16x2_bits(vec_amax2(a), vec_amax2(b)),
+                                                     max_bf16x2_bits(vec_amax2(c), vec_amax2(d))));
+        }
+        for (; v < nvec; v += stride) m2 = max_bf16x2_bits(m2, vec_amax2(ld_v4(row + v * VEC)));
+    }
+    uint32_t m = block_max_u32(hmax_pair(m2), red);
+    if (threadIdx.x == 0) partials[(int64_t)blockIdx.y * gridDim.x + blockIdx.x] = m;
+}
+
+// Phase 2 (current scaling) or the single pass (delayed scaling, t >= 1).
+//   SRC_PARTIALS: s from the phase-1 partials (every CTA reduces them itself, so
+//                 no counter or grid barrier is needed).  When ring != nullptr
+//                 (delayed step 0) CTA 0 also records ring[slot] = amax.
+//   SRC_RING:     s from max(ring); the CTAs also reduce amax_t of this input
+//                 into *pending and the last CTA to finish (ticket) commits it to
+//                 ring[slot] and rearms pending/ticket.
+enum { SRC_PARTIALS = 0, SRC_RING = 1 };
+
+template <int FMT, bool DEQ, int SRC>
+__global__ void __launch_bounds__(QT) cast_tensor_kernel(
+    const uint16_t* __restrict__ x, int64_t nrows, int64_t nvec, int64_t ld,
+    const uint32_t* __restrict__ partials, int32_t npartials,
+    float* ring, int32_t ring_len, int32_t slot, float* pending, uint32_t* ticket,
+    uint8_t* __restrict__ q, float* __restrict__ scale_out, uint16_t* __restrict__ deq,
+    int32_t* status) {
+    __shared__ uint32_t red[32];
+    // ---- the scale
+    uint32_t src = 0;
+    if (SRC == SRC_PARTIALS) {
+        for (int i = threadIdx.x; i < npartials; i += QT) src = max(src, partials[i]);
+    } else {
+        for (int i = threadIdx.x; i < ring_len; i += QT) src = max(src, __float_as_uint(ring[i]));
+    }
+    src = block_max_u32(src, red);
+    float amax;
+    if (SRC == SRC_PARTIALS) {
+        if (src >= 0x7F80u) {
+            if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) report_status(status, FP8_ERR_NONFINITE);
+            src = 0x7F7Fu;     // keep the scale finite; outputs are unspecified then
+        }
+        amax = bf16bits_to_float(src);
+    } else {
+        amax = __uint_as_float(src);
+    }
+    const DivScale op{scale_from_amax<FMT>(amax)};
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        scale_out[0] = op.s;
+        if (SRC == SRC_PARTIALS && ring != nullptr) ring[slot] = amax;
+    }
+    // ---- the cast
+    uint32_t m2 = 0;
+    const int64_t stride = (int64_t)gridDim.x * QT;
+    for (int64_t r = blockIdx.y; r < nrows; r += gridDim.y) {
+        const uint16_t* row = x + r * ld;
+        uint8_t* qrow = q + r * (nvec * VEC);
+        uint16_t* drow = DEQ ? deq + r * (nvec * VEC) : nullptr;
+        int64_t v = (int64_t)blockIdx.x * QT + threadIdx.x;
+        for (; v + stride < nvec; v += 2 * stride) {
+            uint4 a = ld_v4(row + v * VEC);
+            uint4 b = ld_v4(row + (v + stride) * VEC);
+            if (SRC == SRC_RING) m2 = max_bf16x2_bits(m2, max_bf16x2_bits(vec_amax2(a), vec_amax2(b)));
+            uint2 ca = cast_vec<FMT>(a, op), cb = cast_vec<FMT>(b, op);
+            *reinterpret_cast<uint2*>(qrow + v * VEC) = ca;
+            *reinterpret_cast<uint2*>(qrow + (v + stride) * VEC) = cb;
+            if (DEQ) {
+                st_v4_stream(drow + v * VEC, dequant_vec<FMT>(ca, op.s));
+                st_v4_stream(drow + (v + stride) * VEC, dequant_vec<FMT>(cb, op.s));
+            }
+        }
+        for (; v < nvec; v += stride) {
+            uint4 a = ld_v4(row + v * VEC);
+            if (SRC == SRC_RING) m2 = max_bf16x2_bits(m2, vec_amax2(a));
+            uint2 ca = cast_vec<FMT>(a, op);
+            *reinterpret_cast<uint2*>(qrow + v * VEC) = ca;
+            if (DEQ) st_v4_stream(drow + v * VEC, dequant_vec<FMT>(ca, op.s));
+        }
+    }
+    if (SRC == SRC_RING) {
+        uint32_t m = block_max_u32(hmax_pair(m2), red);
+        if (threadIdx.x == 0) {
+            if (m >= 0x7F80u) report_status(status, FP8_ERR_NONFINITE);
+            // amax >= 0, so the fp32 bit pattern orders like the value
+            atomicMax(reinterpret_cast<uint32_t*>(pending), m << 16);
+            __threadfence();
+            const uint32_t total = gridDim.x * gridDim.y;
+            uint32_t t = atomicAdd(ticket, 1u);
+            if (t == total - 1) {
+                // every CTA has read the ring (they all did so before taking a ticket)
+                __threadfence();
+                uint32_t a_t = atomicOr(reinterpret_cast<uint32_t*>(pending), 0u);
+                ring[slot] = __uint_as_float(a_t);
+                *reinterpret_cast<volatile uint32_t*>(pending) = 0u;
+                *reinterpret_cast<volatile uint32_t*>(ticket) = 0u;
+            }
+        }
+    }
+}
+
+// ================================================================ segment kernels
+// ROW (short rows), BLOCK_1x128 and MX32: a group of G lanes (inside one warp)
+// owns one segment (a run of seg_vec vectors of one row) at a time; each lane
+// holds up to U vectors of it in registers, so x is read exactly once.
+//   FLAT: dense tensor whose rows split into whole segments; segment s starts at
+//         element s*seg_vec*8 and owns scale s.
+template <int FMT, bool DEQ, int G, int U, bool MX, bool FLAT>
+__global__ void __launch_bounds__(QT) quant_segment_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    int32_t seg_vec, int64_t nseg_per_row, int64_t nseg,
+    uint8_t* __restrict__ q, void* __restrict__ scale, uint16_t* __restrict__ deq, int32_t* status) {
+    const int lane_g = threadIdx.x & (G - 1);
+    const int64_t group = ((int64_t)blockIdx.x * QT + threadIdx.x) / G;
+    const int64_t ngroups = (int64_t)gridDim.x * (QT / G);
+    const unsigned gmask = G == 32 ? 0xffffffffu : (((1u << G) - 1u) << ((threadIdx.x & 31) & ~(G - 1)));
+    for (int64_t s = group; s < nseg; s += ngroups) {
+        int64_t row, c0;
+        int32_t len_vec;
+        if (FLAT) {
+            row = 0; c0 = s * (int64_t)seg_vec * VEC; len_vec = seg_vec;
+        } else {
+            row = s / nseg_per_row;
+            c0 = (s - row * nseg_per_row) * (int64_t)seg_vec * VEC;
+            int64_t rem = (cols - c0) / VEC;
+            len_vec = rem < seg_vec ? (int32_t)rem : seg_vec;
+        }
+        const uint16_t* src = x + row * ld + c0;
+        uint4 v[U];
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < U; ++i) {
+            const int k = lane_g + G * i;
+            if (k < len_vec) {
+                v[i] = ld_v4_stream(src + (int64_t)k * VEC);
+                m2 = max_bf16x2_bits(m2, vec_amax2(v[i]));
+            }
+        }
+        uint32_t m = hmax_pair(m2);
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(gmask, m, o));
+        if (m >= 0x7F80u) {
+            if (lane_g == 0) report_status(status, FP8_ERR_NONFINITE);
+            m = 0x7F7Fu;
+        }
+        uint8_t* dst = q + row * cols + c0;
+        uint16_t* ddst = DEQ ? deq + row * cols + c0 : nullptr;
+        if (MX) {
+            const int e = mx_exponent(m);
+            const Pow2Scale op{exp2i(-e), exp2i(e)};
+            if (lane_g == 0) reinterpret_cast<uint8_t*>(scale)[s] = (uint8_t)(e + 127);
+#pragma unroll
+            for (int i = 0; i < U; ++i) {
+                const int k = lane_g + G * i;
+                if (k < len_vec) {
+                    uint2 c = cast_vec<FMT>(v[i], op);
+                    *reinterpret_cast<uint2*>(dst + (int64_t)k * VEC) = c;
+                    if (DEQ) st_v4_stream(ddst + (int64_t)k * VEC, dequant_vec<FMT>(c, op.deq()));
+                }
+            }
+        } else {
+            const DivScale op{scale_from_amax<FMT>(bf16bits_to_float(m))};
+            if (lane_g == 0) reinterpret_cast<float*>(scale)[s] = op.s;
+#pragma unroll
+            for (int i = 0; i < U; ++i) {
+                const int k = lane_g + G * i;
+                if (k < len_vec) {
+                    uint2 c = cast_vec<FMT>(v[i], op);
+                    *reinterpret_cast<uint2*>(dst + (int64_t)k * VEC) = c;
+                    if (DEQ) st_v4_stream(ddst + (int64_t)k * VEC, dequant_vec<FMT>(c, op.s));
+                }
+            }
+        }
+    }
+}
+
+// ROW with long rows: one CTA per row.  Rows of up to QT*UR vectors stay in
+// registers (single pass); longer rows take a second pass for the cast.
+template <int FMT, bool DEQ, int UR>
+__global__ void __launch_bounds__(QT) quant_row_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                       int64_t cols, int64_t ld, uint8_t* __restrict__ q,
+                                                       float* __restrict__ scale, uint16_t* __restrict__ deq,
+                                                       int32_t* status) {
+    __shared__ uint32_t red[32];
+    const int64_t nvec = cols / VEC;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const uint16_t* src = x + r * ld;
+        uint4 v[UR];
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < UR; ++i) {
+            const int64_t k = threadIdx.x + (int64_t)QT * i;
+            if (k < nvec) {
+                v[i] = ld_v4_stream(src + k * VEC);
+                m2 = max_bf16x2_bits(m2, vec_amax2(v[i]));
+            }
+        }
+        for (int64_t k = threadIdx.x + (int64_t)QT * UR; k < nvec; k += QT)
+            m2 = max_bf16x2_bits(m2, vec_amax2(ld_v4(src + k * VEC)));
+        uint32_t m = block_max_u32(hmax_pair(m2), red);
+        if (m >= 0x7F80u) {
+            if (threadIdx.x == 0) report_status(status, FP8_ERR_NONFINITE);
+            m = 0x7F7Fu;
+        }
+        const DivScale op{scale_from_amax<FMT>(bf16bits_to_float(m))};
+        if (threadIdx.x == 0) scale[r] = op.s;
+        uint8_t* dst = q + r * cols;
+        uint16_t* ddst = DEQ ? deq + r * cols : nullptr;
+#pragma unroll
+        for (int i = 0; i < UR; ++i) {
+            const int64_t k = threadIdx.x + (int64_t)QT * i;
+            if (k < nvec) {
+                uint2 c = cast_vec<FMT>(v[i], op);
+                *reinterpret_cast<uint2*>(dst + k * VEC) = c;
+                if (DEQ) st_v4_stream(ddst + k * VEC, dequant_vec<FMT>(c, op.s));
+            }
+        }
+        for (int64_t k = threadIdx.x + (int64_t)QT * UR; k < nvec; k += QT) {
+            uint2 c = cast_vec<FMT>(ld_v4(src + k * VEC), op);
+            *reinterpret_cast<uint2*>(dst + k * VEC) = c;
+            if (DEQ) st_v4_stream(ddst + k * VEC, dequant_vec<FMT>(c, op.s));
+        }
+        __syncthreads();   // red[] is reused by the next row
+    }
+}
+
+// BLOCK_128x128: one CTA per 128 x 128 tile; the 2048 vectors of a full tile sit
+// in registers (8 per thread), rows of the tile are read by 16 consecutive lanes.
+template <int FMT, bool DEQ>
+__global__ void __launch_bounds__(QT) quant_block128_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                            int64_t cols, int64_t ld, uint8_t* __restrict__ q,
+                                                            float* __restrict__ scale, uint16_t* __restrict__ deq,
+                                                            int32_t* status) {
+    __shared__ uint32_t red[32];
+    constexpr int UB = 128 * 16 / QT;   // 8 vectors per thread
+    const int64_t ncb = (cols + 127) / 128;
+    const int64_t r0 = (int64_t)blockIdx.y * 128, c0 = (int64_t)blockIdx.x * 128;
+    uint4 v[UB];
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < UB; ++i) {
+        const int idx = threadIdx.x + QT * i;
+        const int64_t r = r0 + (idx >> 4), c = c0 + (idx & 15) * VEC;
+        if (r < rows && c < cols) {
+            v[i] = ld_v4_stream(x + r * ld + c);
+            m2 = max_bf16x2_bits(m2, vec_amax2(v[i]));
+        }
+    }
+    uint32_t m = block_max_u32(hmax_pair(m2), red);
+    if (m >= 0x7F80u) {
+        if (threadIdx.x == 0) report_status(status, FP8_ERR_NONFINITE);
+        m = 0x7F7Fu;
+    }
+    const DivScale op{scale_from_amax<FMT>(bf16bits_to_float(m))};
+    if (threadIdx.x == 0) scale[(int64_t)blockIdx.y * ncb + blockIdx.x] = op.s;
+#pragma unroll
+    for (int i = 0; i < UB; ++i) {
+        const int idx = threadIdx.x + QT * i;
+        const int64_t r = r0 + (idx >> 4), c = c0 + (idx & 15) * VEC;
+        if (r < rows && c < cols) {
+            uint2 cq = cast_vec<FMT>(v[i], op);
+            *reinterpret_cast<uint2*>(q + r * cols + c) = cq;
+            if (DEQ) st_v4_stream(deq + r * cols + c, dequant_vec<FMT>(cq, op.s));
+        }
+    }
+}
+
+// ================================================================ launchers
+static int sm_count_cached() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+int32_t amax_partials_count() { return 148 * 8; }
+
+// Grid for the streaming per-tensor kernels: at most amax_partials_count() CTAs.
+static dim3 tensor_grid(int64_t nrows, int64_t nvec) {
+    const int64_t cap = std::min<int64_t>(amax_partials_count(), (int64_t)sm_count_cached() * 8);
+    int64_t gx = std::max<int64_t>(1, std::min<int64_t>((nvec + QT - 1) / QT, cap));
+    int64_t gy = std::max<int64_t>(1, std::min<int64_t>(nrows, cap / gx));
+    gy = std::min<int64_t>(gy, 65535);
+    return dim3((unsigned)gx, (unsigned)gy);
+}
+
+template <int FMT, bool DEQ>
+static void launch_cast_tensor(const QuantArgs& a, int src, dim3 grid, int npart, float* ring, int32_t len,
+                               int32_t slot, float* pending, uint32_t* ticket, int64_t nrows, int64_t nvec,
+                               int64_t ld, cudaStream_t st) {
+    if (src == SRC_PARTIALS)
+        cast_tensor_kernel<FMT, DEQ, SRC_PARTIALS><<<grid, QT, 0, st>>>(
+            a.x, nrows, nvec, ld, a.partials, npart, ring, len, slot, pending, ticket, a.q,
+            (float*)a.scale, a.deq, a.status);
+    else
+        cast_tensor_kernel<FMT, DEQ, SRC_RING><<<grid, QT, 0, st>>>(
+            a.x, nrows, nvec, ld, a.partials, npart, ring, len, slot, pending, ticket, a.q,
+            (float*)a.scale, a.deq, a.status);
+}
+
+// Per-tensor current scaling (two launches) or one delayed step.
+cudaError_t launch_quantize_tensor(const QuantArgs& a, cudaStream_t st) {
+    const bool dense = a.ld == a.cols;
+    const int64_t nrows = dense ? (a.rows > 0 ? 1 : 0) : a.rows;
+    const int64_t nvec = dense ? a.rows * a.cols / VEC : a.cols / VEC;
+    dim3 grid = tensor_grid(std::max<int64_t>(nrows, 1), std::max<int64_t>(nvec, 1));
+    const int npart = (int)(grid.x * grid.y);
+    const bool delayed_t = a.hist_ring != nullptr && a.hist_step > 0;
+    const int32_t slot = a.hist_ring ? (int32_t)(a.hist_step % a.hist_len) : 0;
+    if (!delayed_t)
+        amax_partials_kernel<<<grid, QT, 0, st>>>(a.x, nrows, nvec, a.ld, a.partials);
+    const int src = delayed_t ? SRC_RING : SRC_PARTIALS;
+    const bool deq = a.deq != nullptr;
+    if (a.fmt == FP8_E4M3) {
+        if (deq) launch_cast_tensor<FP8_E4M3, true>(a, src, grid, npart, a.hist_ring, a.hist_len, slot, a.hist_pending, a.hist_ticket, nrows, nvec, a.ld, st);
+        else     launch_cast_tensor<FP8_E4M3, false>(a, src, grid, npart, a.hist_ring, a.hist_len, slot, a.hist_pending, a.hist_ticket, nrows, nvec, a.ld, st);
+    } else {
+        if (deq) launch_cast_tensor<FP8_E5M2, true>(a, src, grid, npart, a.hist_ring, a.hist_len, slot, a.hist_pending, a.hist_ticket, nrows, nvec, a.ld, st);
+        else     launch_cast_tensor<FP8_E5M2, false>(a, src, grid, npart, a.hist_ring, a.hist_len, slot, a.hist_pending, a.hist_ticket, nrows, nvec, a.ld, st);
+    }
+    return cudaGetLastError();
+}
+
+template <int FMT, bool DEQ, int G, int U, bool MX>
+static void launch_segment(const QuantArgs& a, int32_t seg_vec, cudaStream_t st) {
+    const int64_t seg_elems = (int64_t)seg_vec * VEC;
+    const int64_t nspr = (a.cols + seg_elems - 1) / seg_elems;
+    const int64_t nseg = a.rows * nspr;
+    if (nseg == 0) return;
+    const bool flat = a.ld == a.cols && a.cols % seg_elems == 0;
+    const int64_t groups_needed = nseg;
+    const int64_t cap = (int64_t)sm_count_cached() * 8;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((groups_needed * G + QT - 1) / QT, cap * 16));
+    if (flat)
+        quant_segment_kernel<FMT, DEQ, G, U, MX, true><<<(unsigned)blocks, QT, 0, st>>>(
+            a.x, a.rows, a.cols, a.ld, seg_vec, nspr, nseg, a.q, a.scale, a.deq, a.status);
+    else
+        quant_segment_kernel<FMT, DEQ, G, U, MX, false><<<(unsigned)blocks, QT, 0, st>>>(
+            a.x, a.rows, a.cols, a.ld, seg_vec, nspr, nseg, a.q, a.scale, a.deq, a.status);
+}
+
+template <int FMT, bool DEQ>
+static cudaError_t quantize_grouped_t(const QuantArgs& a, cudaStream_t st) {
+    switch (a.mode) {
+    case FP8_SCALE_ROW: {
+        const int64_t nvec = a.cols / VEC;
+        if (nvec <= 32 * 8) {
+            // short rows: a warp (or less) per row
+            if (nvec <= 4 * 4)       launch_segment<FMT, DEQ, 4, 4, false>(a, (int32_t)nvec, st);
+            else if (nvec <= 16 * 4) launch_segment<FMT, DEQ, 16, 4, false>(a, (int32_t)nvec, st);
+            else                     launch_segment<FMT, DEQ, 32, 8, false>(a, (int32_t)nvec, st);
+        } else {
+            const int64_t blocks = std::min<int64_t>(a.rows, (int64_t)1 << 30);
+            if (nvec <= QT * 4)
+                quant_row_kernel<FMT, DEQ, 4><<<(unsigned)blocks, QT, 0, st>>>(a.x, a.rows, a.cols, a.ld, a.q, (float*)a.scale, a.deq, a.status);
+            else
+                quant_row_kernel<FMT, DEQ, 8><<<(unsigned)blocks, QT, 0, st>>>(a.x, a.rows, a.cols, a.ld, a.q, (float*)a.scale, a.deq, a.status);
+        }
+        break;
+    }
+    case FP8_SCALE_BLOCK_1x128:
+        launch_segment<FMT, DEQ, 4, 4, false>(a, 16, st);
+        break;
+    case FP8_SCALE_MX32:
+        launch_segment<FMT, DEQ, 4, 1, true>(a, 4, st);
+        break;
+    case FP8_SCALE_BLOCK_128x128: {
+        dim3 grid((unsigned)((a.cols + 127) / 128), (unsigned)((a.rows + 127) / 128));
+        if (grid.x && grid.y)
+            quant_block128_kernel<FMT, DEQ><<<grid, QT, 0, st>>>(a.x, a.rows, a.cols, a.ld, a.q, (float*)a.scale, a.deq, a.status);
+        break;
+    }
+    default:
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_grouped(const QuantArgs& a, cudaStream_t st) {
+    const bool deq = a.deq != nullptr;
+    if (a.fmt == FP8_E4M3) return deq ? quantize_grouped_t<FP8_E4M3, true>(a, st) : quantize_grouped_t<FP8_E4M3, false>(a, st);
+    if (a.mode == FP8_SCALE_MX32) return cudaErrorInvalidValue;
+    return deq ? quantize_grouped_t<FP8_E5M2, true>(a, st) : quantize_grouped_t<FP8_E5M2, false>(a, st);
+}
+
+// Scales of empty inputs: amax = 0 gives the floor scale (MX: byte 0).
+__global__ void fill_floor_scale_kernel(float* s, int64_t n, float v) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) s[i] = v;
+}
+
+cudaError_t launch_fill_scale(float* s, int64_t n, float v, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 1024);
+    fill_floor_scale_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, n, v);
+    return cudaGetLastError();
+}
+
+}  // namespace fp8b

@@ -1,0 +1,192 @@
+/*
+ * fp8.h -- C ABI of libfp8.so, the B200 (sm_100a) FP8 runtime linear path.
+ *
+ * The path, as the source pages describe it:
+ *   X --amax reduce--> a_max --scale--> s = a_max / F_max --clip and cast--> X_fp8
+ *   Y = s_x * s_w * (X_fp8 W_fp8^T), FP32 accumulation, BF16 output.
+ * Pages cited below:
+ *   [FFS] "FP8 formats, scaling and LLM inference" (charlestar.github.io)
+ *   [PQG] "FP8 产线量化落地指南" (m.xxqk.cn)
+ *   [FPI] "FP8 推理：8 位浮点量化、E4M3/E5M2 与 NVIDIA FP8 生态" (plumephp.com)
+ *   [FRLP] "41. FP8 Runtime Low Precision Paths" (datawhalechina llm-algo-leetcode)
+ *
+ * Conventions for every entry point
+ *  - Pointers named *_dev are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory on these paths.  `stream` is a cudaStream_t
+ *    (NULL = legacy default stream).  Work is enqueued asynchronously; nothing
+ *    synchronises the host.
+ *  - The returned status reports only the synchronous argument checks and launch
+ *    errors.  Conditions found on the device are written to `dev_status` (a
+ *    device int32 the caller zeroes; nullable): the first error code found is
+ *    stored there, and the caller reads it after synchronising.
+ *  - Layouts are row-major, last index contiguous.  X is [M, K] with row stride
+ *    ld (elements); W is [N, K] (out x in, as nn.Linear stores it); Y = X W^T is
+ *    [M, N] with row stride ldy.
+ *  - Codes are 8-bit E4M3 ("fn": no Inf, NaN = S.1111.111) or E5M2 (IEEE-style
+ *    Inf/NaN) with biases 7 / 15 and maxima 448 / 57344 ([FFS] section
+ *    "8 个 Bit 怎样分配"; [FPI] section "数值特性").
+ *  - Rounding is IEEE round-to-nearest-even everywhere; x/s is an fp32 IEEE
+ *    division; values are clipped to +-F_max before the cast ([PQG] code step 3).
+ *  - Inputs must be finite; a NaN/Inf input sets FP8_ERR_NONFINITE in dev_status
+ *    and leaves the outputs unspecified ([FFS] section "数值验证看什么", non-finite).
+ */
+#ifndef FP8_B200_H
+#define FP8_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP8_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FP8_API __attribute__((visibility("default")))
+#else
+#define FP8_API
+#endif
+
+typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_format_t;
+
+/*
+ * Scaling granularity ([FFS] sections "Per-tensor Scaling 的优点与问题",
+ * "Per-channel 与 Block Scaling", "Current Scaling", "Delayed Scaling").
+ * Scale buffer layout produced by fp8_quantize for a [rows, cols] input:
+ *   TENSOR         float[1]
+ *   ROW            float[rows]                 (per token for X, per output channel for W)
+ *   BLOCK_1x128    float[rows][ceil(cols/128)]  (1 x 128 blocks along the row)
+ *   BLOCK_128x128  float[ceil(rows/128)][ceil(cols/128)]
+ *   MX32           uint8[rows][cols/32], E8M0 (2^(byte-127)), E4M3 codes only
+ *   DELAYED        float[1], from the amax history (see fp8_history_t)
+ * Every float scale is the dequantisation multiplier s = fp32(max(amax, 1e-12f) / F_max)
+ * ([FFS] eq. s = a_max / F_max; [PQG] code: amax floor 1e-12); MX32 stores
+ * e = clamp(floor(log2 amax) - 8, -127, 127) as the byte e + 127 (amax = 0 -> 0).
+ */
+typedef enum {
+    FP8_SCALE_TENSOR = 0,
+    FP8_SCALE_ROW = 1,
+    FP8_SCALE_BLOCK_1x128 = 2,
+    FP8_SCALE_BLOCK_128x128 = 3,
+    FP8_SCALE_MX32 = 4,
+    FP8_SCALE_DELAYED = 5
+} fp8_scaling_t;
+
+typedef enum {
+    FP8_OK = 0,
+    FP8_ERR_INVALID_ARG = 1,        /* a size, mode, format or pointer is invalid */
+    FP8_ERR_ALIGNMENT = 2,          /* a pointer or stride breaks the 16-byte rules */
+    FP8_ERR_UNSUPPORTED_DEVICE = 3, /* the current device is not compute capability 10.x */
+    FP8_ERR_NONFINITE = 4,          /* (dev_status) a NaN/Inf input element was seen */
+    FP8_ERR_TIMEOUT = 5,            /* (dev_status) a bounded device-side wait gave up */
+    FP8_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed */
+    FP8_ERR_WORKSPACE = 7           /* workspace missing or smaller than fp8_workspace_size() */
+} fp8_status_t;
+
+/*
+ * Amax history for delayed scaling ([FFS] section "Delayed Scaling":
+ * s_{t+1} = f(a_t, ..., a_{t-h+1}) / F_max, with f = window maximum).
+ *   ring_dev     float[len] on the device, zero before step 0.
+ *   len          window length h (>= 1).
+ *   step         host-side step counter t; fp8_quantize reads it and adds 1 after
+ *                enqueueing the step.
+ *   pending_dev  one device float, zero before step 0 (running amax of the step).
+ *   ticket_dev   one device uint32, zero before step 0 (CTA arrival counter).
+ * Step 0 has no history and uses current per-tensor scaling; step t >= 1 uses
+ * s_t = max(max(ring), 1e-12f) / F_max.  After the step, ring[t mod h] holds the
+ * raw amax of X_t, and pending/ticket are back to zero.  Two steps on the same
+ * history must be stream-ordered.
+ */
+typedef struct {
+    float* ring_dev;
+    int32_t len;
+    int64_t step;
+    float* pending_dev;
+    uint32_t* ticket_dev;
+} fp8_history_t;
+
+/* ABI version (FP8_ABI_VERSION). */
+FP8_API int32_t fp8_abi_version(void);
+
+/* Human-readable name of a status code (static storage). */
+FP8_API const char* fp8_status_string(int32_t status);
+
+/* FP8_OK when the current CUDA device is compute capability 10.x (sm_100a),
+ * FP8_ERR_UNSUPPORTED_DEVICE otherwise, FP8_ERR_CUDA when CUDA is unusable.
+ * (The device gate of [FRLP] section "5.2" preflight, moved to the library.) */
+FP8_API int32_t fp8_device_check(void);
+
+/*
+ * Workspace bytes an entry point needs.  which: 0 = fp8_quantize,
+ * 1 = fp8_scaled_gemm, 2 = fp8_linear_forward.  For 0, (M, K) is the input
+ * shape [rows, cols] and N is ignored.  The workspace needs no initialisation
+ * and holds nothing between calls.
+ */
+FP8_API size_t fp8_workspace_size(int32_t which, int64_t M, int64_t N, int64_t K, int32_t mode);
+
+/*
+ * fp8_quantize -- amax reduce + scale + clip + RNE cast (+ optional dequant).
+ * [FFS] section "Scale 怎样把 Tensor 塞进 E4M3": X_fp8 = cast(clip(X / s)),
+ * a_max = max|X|, s = a_max / F_max, X^ = s X_fp8; [PQG] section
+ * "运行时动态张量缩放" and its code fp8_dynamic_quantize_tensor.
+ *   x_dev        bf16 [rows, cols], row stride ld elements.  16-byte aligned, ld % 8 == 0.
+ *   rows, cols   >= 0; cols % 16 == 0 (cols % 32 == 0 for MX32).  rows == 0 or
+ *                cols == 0 still writes the scales (amax = 0 -> floor scale).
+ *   fmt          FP8_E4M3 or FP8_E5M2 (MX32: E4M3 only).
+ *   mode         fp8_scaling_t; DELAYED needs hist.
+ *   q_dev        uint8 codes [rows, cols], dense (row stride cols), 16-byte aligned.
+ *   scale_dev    scale buffer in the layout listed with fp8_scaling_t.
+ *   hist         host struct, DELAYED only (else NULL); its step is advanced.
+ *   dequant_dev  nullable; bf16 [rows, cols] dense, bf16_RNE(fp32(decode(q) * s)).
+ *   dev_status   nullable device int32 (FP8_ERR_NONFINITE).
+ *   workspace_dev, ws_bytes  at least fp8_workspace_size(0, rows, 0, cols, mode) bytes
+ *                (0 for modes other than TENSOR/DELAYED).
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, WORKSPACE, CUDA.
+ */
+FP8_API int32_t fp8_quantize(const void* x_dev, int64_t rows, int64_t cols, int64_t ld,
+                     int32_t fmt, int32_t mode, uint8_t* q_dev, void* scale_dev,
+                     fp8_history_t* hist, void* dequant_dev, int32_t* dev_status,
+                     void* workspace_dev, size_t ws_bytes, void* stream);
+
+/*
+ * fp8_scaled_gemm -- Y = bf16( sum_k S_a(m,k) a[m,k] * S_b(n,k) b[n,k] ) with FP32
+ * accumulation on the tcgen05 tensor cores ([FFS] section
+ * "一次 FP8 GEMM 的完整精度契约": Y ~= s_x s_w (X_8 W_8), wider accumulation,
+ * BF16 output; [PQG] code fp8_gemm_forward, out_dtype bf16).
+ *   a_dev [M, K] and b_dev [N, K]: codes, dense row-major (K contiguous), 16-byte aligned.
+ *   a_scale_dev / b_scale_dev in the fp8_quantize layout for a_mode / b_mode.
+ *   Mode pairs: a, b in {TENSOR, ROW, DELAYED} (DELAYED reads as TENSOR), any
+ *   mix; (BLOCK_1x128, BLOCK_128x128); (MX32, MX32).
+ *   fmt_a, fmt_b: E4M3 or E5M2 for the tensor/row modes; E4M3 for block and MX32.
+ *   K % 16 == 0 (K % 32 == 0 for MX32); M, N >= 0; K == 0 writes zeros.
+ *   y_dev bf16 [M, N], row stride ldy (ldy % 8 == 0, ldy >= N), 16-byte aligned.
+ *   dev_status: nullable device int32; FP8_ERR_TIMEOUT if a pipeline wait gave up.
+ * The workspace is unused (pass NULL, 0).
+ */
+FP8_API int32_t fp8_scaled_gemm(const uint8_t* a_dev, const void* a_scale_dev, int32_t a_mode, int32_t fmt_a,
+                        const uint8_t* b_dev, const void* b_scale_dev, int32_t b_mode, int32_t fmt_b,
+                        int64_t M, int64_t N, int64_t K, void* y_dev, int64_t ldy,
+                        int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream);
+
+/*
+ * fp8_linear_forward -- one FP8 linear layer: quantize X with x_mode (current
+ * scaling, or DELAYED with hist) into the workspace, then fp8_scaled_gemm with
+ * the pre-quantised static weight ([PQG] section "运行时动态张量缩放": S_w fixed
+ * offline, S_x computed per batch on the GPU; [FFS] section "Weight Scale 与
+ * Activation Scale 生命周期不同").
+ *   x_dev bf16 [M, K], row stride ldx.  x_mode: TENSOR, ROW, BLOCK_1x128, MX32
+ *   or DELAYED; w_mode must pair with it as in fp8_scaled_gemm.
+ *   w_dev/w_scale_dev: codes [N, K] and scales as fp8_quantize produced them.
+ *   workspace: fp8_workspace_size(2, M, N, K, x_mode) bytes, 256-byte aligned.
+ */
+FP8_API int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt,
+                           int32_t x_mode, fp8_history_t* hist,
+                           const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
+                           int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy,
+                           int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8_B200_H */
