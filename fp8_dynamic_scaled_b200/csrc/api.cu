@@ -55,7 +55,7 @@ int32_t check_quantize_args(const void* x, int64_t rows, int64_t cols, int64_t l
     if (rows >= ((int64_t)1 << 40) || cols >= ((int64_t)1 << 40)) return FP8_ERR_INVALID_ARG;
     if (cols % 16 != 0) return FP8_ERR_INVALID_ARG;
     if (mode == FP8_SCALE_MX32 && cols % 32 != 0) return FP8_ERR_INVALID_ARG;
-    if (scale == nullptr) return FP8_ERR_INVALID_ARG;
+    if (scale == nullptr && scale_bytes(mode, rows, cols) > 0) return FP8_ERR_INVALID_ARG;
     const bool empty = rows == 0 || cols == 0;
     if (!empty && (x == nullptr || q == nullptr)) return FP8_ERR_INVALID_ARG;
     if (mode == FP8_SCALE_DELAYED) {
@@ -127,8 +127,7 @@ int32_t check_gemm_args(const uint8_t* a, const void* sa, int32_t am, int32_t fa
         if (y == nullptr) return FP8_ERR_INVALID_ARG;
         if (K > 0 && (a == nullptr || b == nullptr || sa == nullptr || sb == nullptr)) return FP8_ERR_INVALID_ARG;
     }
-    if (ldy % 8 != 0) return FP8_ERR_ALIGNMENT;
-    if (!aligned16(a) || !aligned16(b) || !aligned16(y)) return FP8_ERR_ALIGNMENT;
+    if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(y) & 1u) != 0) return FP8_ERR_ALIGNMENT;
     if (!mx && (((reinterpret_cast<uintptr_t>(sa) | reinterpret_cast<uintptr_t>(sb)) & 3u) != 0)) return FP8_ERR_ALIGNMENT;
     return FP8_OK;
 }

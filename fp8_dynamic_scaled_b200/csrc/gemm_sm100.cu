@@ -26,6 +26,7 @@
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA raises an abort
 // flag, reports FP8_ERR_TIMEOUT in dev_status, drains and frees TMEM, and exits.
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -94,6 +95,11 @@ struct GemmParams {
     const uint8_t* sfb;
     uint32_t idesc;
     int32_t* status;
+    // output written with plain stores when it cannot be described to TMA
+    // (row stride not a multiple of 16 bytes, or a base address off 16 bytes)
+    uint16_t* y;
+    int64_t ldy;
+    int32_t y_direct;
 };
 
 // ---------------------------------------------------------------- bounded waits
@@ -131,7 +137,20 @@ __device__ __forceinline__ void stage_row_sw64(uint8_t* buf, int r, const uint32
 
 // Store a 32-row x 32-column bf16 chunk held one row per lane.
 __device__ __forceinline__ void store_chunk(const CUtensorMap* tmY, uint8_t* buf, const uint32_t (&w)[16],
-                                            int32_t x, int32_t y, int lane) {
+                                            int32_t x, int32_t y, int lane, const GemmParams& p) {
+    if (p.y_direct) {
+        const int32_t row = y + lane;
+        if (row < p.M) {
+            uint16_t* dst = p.y + (int64_t)row * p.ldy;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int32_t n = x + 2 * j;
+                if (n < p.N) dst[n] = (uint16_t)(w[j] & 0xFFFFu);
+                if (n + 1 < p.N) dst[n + 1] = (uint16_t)(w[j] >> 16);
+            }
+        }
+        return;
+    }
     stage_row_sw64(buf, lane, w);
     ptx::fence_proxy_async_smem();
     __syncwarp();
@@ -180,7 +199,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmA);
         ptx::prefetch_tmap(&tmB);
-        ptx::prefetch_tmap(&tmY);
+        if (!p.y_direct) ptx::prefetch_tmap(&tmY);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -358,7 +377,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
                         __syncwarp();
-                        store_chunk(&tmY, b, w, n0, y_row0, lane);
+                        store_chunk(&tmY, b, w, n0, y_row0, lane, p);
                         ++store_it;
                     }
                 }
@@ -403,7 +422,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
                         __syncwarp();
-                        store_chunk(&tmY, b, w, n0, y_row0, lane);
+                        store_chunk(&tmY, b, w, n0, y_row0, lane, p);
                         ++store_it;
                     }
                 }
@@ -430,7 +449,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
                         __syncwarp();
-                        store_chunk(&tmY, b, w, n0, y_row0, lane);
+                        store_chunk(&tmY, b, w, n0, y_row0, lane, p);
                         ++store_it;
                     }
                 }
@@ -496,9 +515,11 @@ static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaSt
     if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.K, BK, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, BN,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, (uint64_t)g.N, (uint64_t)g.M,
-                     (uint64_t)g.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    memset(&ty, 0, sizeof(ty));
+    if (!p.y_direct && !make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, (uint64_t)g.N, (uint64_t)g.M,
+                                    (uint64_t)g.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     static bool attr_done = false;
     if (!attr_done) {
@@ -537,6 +558,9 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
     // keep the operand with the smaller footprint resident in L2: walk its tiles fastest
     p.m_fastest = (g.M <= g.N) ? 1 : 0;
     p.status = g.status;
+    p.y = g.y;
+    p.ldy = g.ldy;
+    p.y_direct = (g.ldy % 8 != 0 || (reinterpret_cast<uintptr_t>(g.y) & 15u) != 0) ? 1 : 0;
     const bool a_pt = g.a_mode == FP8_SCALE_TENSOR || g.a_mode == FP8_SCALE_DELAYED;
     const bool b_pt = g.b_mode == FP8_SCALE_TENSOR || g.b_mode == FP8_SCALE_DELAYED;
     if ((a_pt || g.a_mode == FP8_SCALE_ROW) && (b_pt || g.b_mode == FP8_SCALE_ROW)) {

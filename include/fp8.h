@@ -160,7 +160,8 @@ FP8_API int32_t fp8_quantize(const void* x_dev, int64_t rows, int64_t cols, int6
  *   mix; (BLOCK_1x128, BLOCK_128x128); (MX32, MX32).
  *   fmt_a, fmt_b: E4M3 or E5M2 for the tensor/row modes; E4M3 for block and MX32.
  *   K % 16 == 0 (K % 32 == 0 for MX32); M, N >= 0; K == 0 writes zeros.
- *   y_dev bf16 [M, N], row stride ldy (ldy % 8 == 0, ldy >= N), 16-byte aligned.
+ *   y_dev bf16 [M, N], row stride ldy >= N.  With ldy % 8 == 0 and a 16-byte aligned
+ *   y_dev the tiles leave through TMA stores; otherwise through plain stores.
  *   dev_status: nullable device int32; FP8_ERR_TIMEOUT if a pipeline wait gave up.
  * The workspace is unused (pass NULL, 0).
  */

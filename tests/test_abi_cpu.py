@@ -75,7 +75,7 @@ def test_argument_validation_without_device(lib):
     assert L.fp8_scaled_gemm(P, P, 2, 0, P, P, 1, 0, 16, 16, 32, P, 16, None, None, 0, None) == b.FP8_ERR_INVALID_ARG
     assert L.fp8_scaled_gemm(P, P, 4, 0, P, P, 4, 1, 16, 16, 32, P, 16, None, None, 0, None) == b.FP8_ERR_INVALID_ARG
     assert L.fp8_scaled_gemm(P, P, 1, 0, P, P, 1, 0, 16, 16, 32, P, 12, None, None, 0, None) == b.FP8_ERR_INVALID_ARG
-    assert L.fp8_scaled_gemm(P, P, 1, 0, P, P, 1, 0, 16, 16, 32, P, 20, None, None, 0, None) == b.FP8_ERR_ALIGNMENT
+    assert L.fp8_scaled_gemm(P, P, 1, 0, P, P, 1, 0, 16, 16, 32, P + 1, 20, None, None, 0, None) == b.FP8_ERR_ALIGNMENT
     # linear forward: workspace missing / too small
     assert L.fp8_linear_forward(P, 16, 32, 32, 0, 1, None, P, P, 1, 0, 16, P, 16, None, None, 0, None) \
         == b.FP8_ERR_WORKSPACE
