@@ -30,7 +30,8 @@ FP8_OK, FP8_ERR_INVALID_ARG, FP8_ERR_ALIGNMENT, FP8_ERR_UNSUPPORTED_DEVICE = 0, 
 FP8_ERR_NONFINITE, FP8_ERR_TIMEOUT, FP8_ERR_CUDA, FP8_ERR_WORKSPACE = 4, 5, 6, 7
 
 EXPORTED = ("fp8_abi_version", "fp8_status_string", "fp8_device_check", "fp8_workspace_size",
-            "fp8_quantize", "fp8_scaled_gemm", "fp8_linear_forward")
+            "fp8_quantize", "fp8_scaled_gemm", "fp8_linear_forward", "fp8_linear_forward_noalloc")
+FP8_NOALLOC_SCRATCH_BYTES = 4194304
 
 
 class fp8_history_t(ctypes.Structure):
@@ -53,6 +54,9 @@ _lib.fp8_scaled_gemm.argtypes = [_P, _P, _I32, _I32, _P, _P, _I32, _I32, _I64, _
 _lib.fp8_linear_forward.restype = _I32
 _lib.fp8_linear_forward.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P, _P,
                                     _I32, _I32, _I64, _P, _I64, _P, _P, _SZ, _P]
+_lib.fp8_linear_forward_noalloc.restype = _I32
+_lib.fp8_linear_forward_noalloc.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P,
+                                            _P, _I32, _I32, _I64, _P, _I64, _P, _P]
 
 
 class FP8Error(RuntimeError):
@@ -160,6 +164,24 @@ def fp8_linear_forward(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, workspace
                                  w_mode, w_fmt, N, _ptr(y), ldy, _ptr(dev_status), _ptr(workspace),
                                  _nbytes(workspace), _stream(stream))
     _check(rc, "fp8_linear_forward")
+
+
+def fp8_linear_forward_noalloc(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, *, hist: History | None = None,
+                               dev_status=None, stream=None):
+    """fp8_linear_forward without a workspace argument, for callers that cannot allocate:
+    the scratch is the library's fixed FP8_NOALLOC_SCRATCH_BYTES device array, shared by
+    all calls (order overlapping calls on one stream)."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.uint8 or y.dtype != torch.bfloat16:
+        raise TypeError("x bf16, w uint8 codes, y bf16")
+    M, K = x.shape
+    N = w.shape[0]
+    ldx = x.stride(0) if M > 1 else K
+    ldy = y.stride(0) if y.shape[0] > 1 else y.shape[1]
+    rc = _lib.fp8_linear_forward_noalloc(_ptr(x), M, K, ldx, x_fmt, x_mode,
+                                         ctypes.byref(hist.c) if hist is not None else None, _ptr(w),
+                                         _ptr(w_scale), w_mode, w_fmt, N, _ptr(y), ldy, _ptr(dev_status),
+                                         _stream(stream))
+    _check(rc, "fp8_linear_forward_noalloc")
 
 
 # ------------------------------------------------------------------ allocation helpers

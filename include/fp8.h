@@ -187,6 +187,38 @@ FP8_API int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int6
                            int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy,
                            int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream);
 
+/*
+ * fp8_linear_forward_noalloc -- fp8_linear_forward for callers that cannot
+ * allocate device memory.  (The source pages have no counterpart: this is a
+ * deployment convenience of this library, not part of the method.)
+ *
+ * Some callers have no way to obtain a workspace: code running inside a host
+ * program that owns all device memory and passes its plug-ins only their input
+ * and output buffers, or code that must not call cudaMalloc because it can
+ * synchronise the whole device.  This entry point takes the same arguments as
+ * fp8_linear_forward except the workspace; its scratch (quantised X, X scales,
+ * per-tensor amax partials) is a fixed array of FP8_NOALLOC_SCRATCH_BYTES of
+ * device memory inside libfp8.so, present on every GPU that loads the library
+ * until the process exits.  The call itself allocates nothing.
+ *   - Size limit: fp8_workspace_size(2, M, N, K, x_mode) must not exceed
+ *     FP8_NOALLOC_SCRATCH_BYTES (e.g. M*K up to ~4.1 million codes); larger
+ *     inputs return FP8_ERR_WORKSPACE and enqueue nothing.
+ *   - The first call on each device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one scratch array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose work can
+ *     overlap on the GPU -- different streams, or unordered host threads -- race
+ *     on it: order them on one stream.
+ * Other arguments, errors and results: as fp8_linear_forward.
+ */
+#define FP8_NOALLOC_SCRATCH_BYTES 4194304
+FP8_API int32_t fp8_linear_forward_noalloc(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt,
+                                           int32_t x_mode, fp8_history_t* hist,
+                                           const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
+                                           int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy,
+                                           int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
