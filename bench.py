@@ -505,7 +505,7 @@ def run_quant_sweep(args, torch, fp8, stream, barrier, dist, world, rank, gpu_in
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama70b_prefill", choices=sorted(WORKLOADS) + ["quant_sweep"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
@@ -557,21 +557,26 @@ def main():
     q_avg = statistics.mean(q_ms)
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_OVER_BF16
     gemm_tflops = flops / (g_avg * 1e-3) / 1e12
-    traffic = profiled_traffic(f"gemm_rowscale_{args.workload}")
-    xbytes = M * K * 3 + 4 * M
+    variant = {1: "ROWSCALE", 2: "BLOCK", 4: "MX"}[wl["x_mode"]]
+    traffic = profiled_traffic(f"gemm_{variant.lower()}_{args.workload}")
+    xbytes = M * K * 3 + {1: 4 * M, 2: 4 * M * (-(-K // 128)), 4: M * (K // 32)}[wl["x_mode"]]
+    qkernel = {1: "stream_quant_kernel<ROW>", 2: "stream_quant_kernel<B128>", 4: "stream_quant_kernel<MX>"}[wl["x_mode"]]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": args.workload, "M": M, "N": N, "K": K, "x_scaling": "per-token",
-                   "w_scaling": "per-channel", "fp8": "e4m3", "out": "bf16",
-                   "l2": "inputs larger than L2 (each step reads 64 MB X + 235 MB W codes, writes 235 MB Y)"},
+        "config": {"workload": args.workload, "M": M, "N": N, "K": K,
+                   "x_scaling": {1: "per-token", 2: "1x128 blocks", 4: "MX32"}[wl["x_mode"]],
+                   "w_scaling": {1: "per-channel", 3: "128x128 blocks", 4: "MX32"}[wl["w_mode"]],
+                   "fp8": "e4m3", "out": "bf16",
+                   "l2": f"inputs larger than L2 (each step reads {2 * M * K / 1e6:.0f} MB X + "
+                         f"{N * K / 1e6:.0f} MB W codes, writes {2 * M * N / 1e6:.0f} MB Y)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": sustained, "unit": "TFLOP/s",
                      "frac": gemm_tflops / sustained, "traffic": traffic,
-                     "kernel": "fp8_gemm_kernel<ROWSCALE>",
+                     "kernel": f"fp8_gemm_kernel<{variant}>",
                      "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16} (fp8/bf16 nominal ratio)",
                      "gemm_us_avg": g_avg * 1e3},
-        "quantize": {"kernel": "quant_row_kernel", "us_avg": q_avg * 1e3, "algorithmic_bytes": xbytes,
+        "quantize": {"kernel": qkernel, "us_avg": q_avg * 1e3, "algorithmic_bytes": xbytes,
                      "GB_per_s": xbytes / (q_avg * 1e-3) / 1e9,
                      "frac_of_hbm": xbytes / (q_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "share_of_gemm_time": q_avg / g_avg},

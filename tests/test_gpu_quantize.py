@@ -85,9 +85,10 @@ def test_quantize_small_shapes(fmt, mode, shape):
 
 
 @pytest.mark.parametrize("mode", MODES)
-def test_quantize_strided_rows(mode):
-    x = mixed_input(200, 512, seed=5)
-    check_parity(x, fp8.FP8_E4M3, mode, ld=512 + 72, what=f"strided mode {mode}")
+@pytest.mark.parametrize("cols", [512, 2048])
+def test_quantize_strided_rows(mode, cols):
+    x = mixed_input(200, cols, seed=5)
+    check_parity(x, fp8.FP8_E4M3, mode, ld=cols + 72, what=f"strided mode {mode}")
 
 
 @pytest.mark.parametrize("mode", MODES)
@@ -116,9 +117,10 @@ def test_quantize_empty(mode):
                               rs.view(np.uint32) if rs.dtype == np.float32 else rs)
 
 
-def test_quantize_nonfinite_sets_status():
+@pytest.mark.parametrize("cols", [256, 2048])
+def test_quantize_nonfinite_sets_status(cols):
     for mode in MODES:
-        x = mixed_input(32, 256, seed=3)
+        x = mixed_input(32, cols, seed=3)
         x[5, 17] = 0x7F80   # +inf
         _, _, _, st = run_gpu(x, fp8.FP8_E4M3, mode)
         assert st == fp8.FP8_ERR_NONFINITE, (mode, st)
@@ -144,14 +146,12 @@ def test_quantize_bad_arguments_rejected():
     assert e.value.status == fp8.FP8_ERR_INVALID_ARG
 
 
-def test_cast_sweep_every_bf16_pattern_many_scales():
-    """Every finite bf16 magnitude below a row's amax, under 2048 different row
-    scales (ROW mode), for both formats: about 65M (x, s) pairs per format."""
-    g = np.random.default_rng(99)
-    pats = np.arange(0, 0x7F80, dtype=np.uint32)                  # finite non-negative bf16 patterns
-    rows = 2048
-    amax_pat = g.integers(0x3000, 0x7F7F, rows).astype(np.uint32)  # amax ~ 1e-10 .. 3e38
-    cols = 32640                                                   # 0x7F80 rounded to a multiple of 16
+def _sweep_input(rows, cols, seed):
+    """Rows whose elements are drawn from every finite bf16 magnitude below a random
+    per-row amax (placed last in the row), with random signs."""
+    g = np.random.default_rng(seed)
+    pats = np.arange(0, 0x7F80, dtype=np.uint32)
+    amax_pat = g.integers(0x3000, 0x7F7F, rows).astype(np.uint32)   # amax ~ 1e-10 .. 3e38
     x = np.zeros((rows, cols), np.uint16)
     for r in range(rows):
         below = pats[pats < amax_pat[r]]
@@ -159,8 +159,24 @@ def test_cast_sweep_every_bf16_pattern_many_scales():
         sign = g.integers(0, 2, cols - 1).astype(np.uint32) << 15
         x[r, :cols - 1] = (pick | sign).astype(np.uint16)
         x[r, cols - 1] = amax_pat[r]
+    return x
+
+
+@pytest.mark.parametrize("mode", [fp8.FP8_SCALE_ROW, fp8.FP8_SCALE_BLOCK_1x128])
+def test_cast_sweep_every_bf16_pattern_many_scales(mode):
+    """Bf16 patterns of every magnitude under thousands of scales (one per row, or one
+    per 1x128 block): about 67M (x, s) pairs per format through the division and the
+    RNE cast, codes and dequant compared bit for bit."""
+    x = _sweep_input(4096, 16384, seed=99 + mode)
     for fmt in FMTS:
-        check_parity(x, fmt, fp8.FP8_SCALE_ROW, dequant=True, what=f"cast sweep fmt {fmt}")
+        check_parity(x, fmt, mode, dequant=True, what=f"cast sweep mode {mode} fmt {fmt}")
+
+
+def test_cast_sweep_long_rows_fallback():
+    """Rows longer than the streaming kernel takes (second-pass row kernel)."""
+    x = _sweep_input(512, 32640, seed=7)
+    for fmt in FMTS:
+        check_parity(x, fmt, fp8.FP8_SCALE_ROW, dequant=True, what=f"long-row sweep fmt {fmt}")
 
 
 # ---------------------------------------------------------------- delayed scaling
