@@ -53,7 +53,8 @@ template <> struct Cfg<V_ROWSCALE> {
     static constexpr uint32_t TMEM_COLS = 512;
 };
 template <> struct Cfg<V_BLOCK> {
-    static constexpr int EPI_WARPS = 8, FIRST_EPI_WARP = 2, STAGE_BUFS = 2;
+    // warps 0-3 (TMA, MMA, two idle) give registers to the 8 epilogue warps (4-11)
+    static constexpr int EPI_WARPS = 8, FIRST_EPI_WARP = 4, STAGE_BUFS = 2;
     static constexpr int ACC_BUFS = 2;            // per-K-block partial products
     static constexpr uint32_t TMEM_COLS = 512;
 };
@@ -86,6 +87,7 @@ struct GemmParams {
     int32_t M, N, K;
     int32_t num_m, num_n, num_kb;
     int32_t m_fastest;
+    int32_t group;          // tiles of the fast dimension per raster group
     // ROWSCALE: element scale = sa[m * sa_stride] * sb[n * sb_stride]
     const float* sa;
     const float* sb;
@@ -120,9 +122,20 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
     }
 }
 
+// Tile raster: the operand with the smaller footprint is walked fastest, in groups
+// of `group` tiles whose panels fit comfortably in L2; within a group the fast index
+// varies fastest and the group sweeps the whole slow dimension before the next group.
 __device__ __forceinline__ void tile_coords(const GemmParams& p, int32_t t, int32_t& mb, int32_t& nb) {
-    if (p.m_fastest) { mb = t % p.num_m; nb = t / p.num_m; }
-    else             { nb = t % p.num_n; mb = t / p.num_n; }
+    const int32_t nfast = p.m_fastest ? p.num_m : p.num_n;
+    const int32_t nslow = p.m_fastest ? p.num_n : p.num_m;
+    const int32_t per_group = p.group * nslow;
+    const int32_t g = t / per_group;
+    const int32_t rem = t - g * per_group;
+    const int32_t width = min(p.group, nfast - g * p.group);
+    const int32_t fast = g * p.group + rem % width;
+    const int32_t slow = rem / width;
+    if (p.m_fastest) { mb = fast; nb = slow; }
+    else             { nb = fast; mb = slow; }
 }
 
 // Write 32 bf16 (16 packed words) of one row into a 32x32 staging tile laid out
@@ -209,7 +222,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-
+    // BLOCK: 384 threads launch with 168 registers each (64,512); warpgroup 0 (TMA,
+    // MMA, two idle warps) keeps 32, the two epilogue warpgroups take 224:
+    // 128*32 + 256*224 = 61,440 <= 64,512, and per SM sub-partition
+    // 32*(32+224+224) = 15,360 <= 16,384.
+    if (warp < C::FIRST_EPI_WARP) {
+    if (V == V_BLOCK) ptx::regs_dec<32>();
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -299,43 +317,90 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         bool ok = true;
         const int32_t kg = p.K / 32;                 // scale bytes per row
         const bool aligned4 = (kg % 4) == 0 && ((reinterpret_cast<uintptr_t>(p.sfa) | reinterpret_cast<uintptr_t>(p.sfb)) & 3u) == 0;
-        for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            int32_t mb, nb;
-            tile_coords(p, t, mb, nb);
-            for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-                uint32_t w[12];
+        // Fast path: 16 scale bytes (four 128-wide stages) per row in one load, the
+        // next group of four fetched while the current one is written out.
+        const bool vec16 = (kg % 16) == 0 && ((reinterpret_cast<uintptr_t>(p.sfa) | reinterpret_cast<uintptr_t>(p.sfb)) & 15u) == 0;
+        auto put_stage = [&](uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t w4, uint32_t w5,
+                             uint32_t w6, uint32_t w7, uint32_t w8, uint32_t w9, uint32_t w10, uint32_t w11) -> bool {
+            if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) return false;
+            uint8_t* dst = sSF + stage * SF_STAGE_BYTES;
+            *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(w0, w1, w2, w3);
+            *reinterpret_cast<uint4*>(dst + 512 + lane * 16) = make_uint4(w4, w5, w6, w7);
+            *reinterpret_cast<uint4*>(dst + 1024 + lane * 16) = make_uint4(w8, w9, w10, w11);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&full[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            return true;
+        };
+        if (vec16) {
+            const int32_t groups = p.num_kb / 4;     // num_kb = 4 * groups here
+            auto load_group = [&](int32_t t, int32_t g, uint4 (&v)[12]) {
+                int32_t mb, nb;
+                tile_coords(p, t, mb, nb);
 #pragma unroll
                 for (int q = 0; q < 12; ++q) {
                     const bool isA = q < 4;
                     const int32_t row = isA ? mb * BM + lane + 32 * q : nb * BN + lane + 32 * (q - 4);
                     const int32_t rows = isA ? p.M : p.N;
                     const uint8_t* base = isA ? p.sfa : p.sfb;
-                    uint32_t v = 0x7F7F7F7Fu;      // 2^0 for rows past the edge (their codes are 0)
-                    if (row < rows) {
-                        const uint8_t* src = base + (int64_t)row * kg + kb * 4;
-                        if (aligned4 && kb * 4 + 4 <= kg) {
-                            v = __ldg(reinterpret_cast<const uint32_t*>(src));
-                        } else {
-                            v = 0;
-                            for (int j = 0; j < 4; ++j)
-                                v |= (uint32_t)(kb * 4 + j < kg ? __ldg(src + j) : 0x7Fu) << (8 * j);
-                        }
-                    }
-                    w[q] = v;
+                    v[q] = row < rows ? __ldg(reinterpret_cast<const uint4*>(base + (int64_t)row * kg + g * 16))
+                                      : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
                 }
-                if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-                uint8_t* dst = sSF + stage * SF_STAGE_BYTES;
-                *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(dst + 512 + lane * 16) = make_uint4(w[4], w[5], w[6], w[7]);
-                *reinterpret_cast<uint4*>(dst + 1024 + lane * 16) = make_uint4(w[8], w[9], w[10], w[11]);
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&full[stage]);
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            };
+            uint4 cur[12], nxt[12];
+            int32_t t = blockIdx.x, g = 0;
+            if (t < num_tiles) load_group(t, 0, cur);
+            while (t < num_tiles && ok) {
+                int32_t tn = t, gn = g + 1;
+                if (gn == groups) { gn = 0; tn = t + gridDim.x; }
+                if (tn < num_tiles) load_group(tn, gn, nxt);
+                ok = put_stage(cur[0].x, cur[1].x, cur[2].x, cur[3].x, cur[4].x, cur[5].x, cur[6].x, cur[7].x,
+                               cur[8].x, cur[9].x, cur[10].x, cur[11].x) &&
+                     put_stage(cur[0].y, cur[1].y, cur[2].y, cur[3].y, cur[4].y, cur[5].y, cur[6].y, cur[7].y,
+                               cur[8].y, cur[9].y, cur[10].y, cur[11].y) &&
+                     put_stage(cur[0].z, cur[1].z, cur[2].z, cur[3].z, cur[4].z, cur[5].z, cur[6].z, cur[7].z,
+                               cur[8].z, cur[9].z, cur[10].z, cur[11].z) &&
+                     put_stage(cur[0].w, cur[1].w, cur[2].w, cur[3].w, cur[4].w, cur[5].w, cur[6].w, cur[7].w,
+                               cur[8].w, cur[9].w, cur[10].w, cur[11].w);
+#pragma unroll
+                for (int q = 0; q < 12; ++q) cur[q] = nxt[q];
+                t = tn;
+                g = gn;
+            }
+        } else {
+            for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                int32_t mb, nb;
+                tile_coords(p, t, mb, nb);
+                for (int32_t kb = 0; kb < p.num_kb && ok; ++kb) {
+                    uint32_t w[12];
+#pragma unroll
+                    for (int q = 0; q < 12; ++q) {
+                        const bool isA = q < 4;
+                        const int32_t row = isA ? mb * BM + lane + 32 * q : nb * BN + lane + 32 * (q - 4);
+                        const int32_t rows = isA ? p.M : p.N;
+                        const uint8_t* base = isA ? p.sfa : p.sfb;
+                        uint32_t v = 0x7F7F7F7Fu;      // 2^0 for rows past the edge (their codes are 0)
+                        if (row < rows) {
+                            const uint8_t* src = base + (int64_t)row * kg + kb * 4;
+                            if (aligned4 && kb * 4 + 4 <= kg) {
+                                v = __ldg(reinterpret_cast<const uint32_t*>(src));
+                            } else {
+                                v = 0;
+                                for (int j = 0; j < 4; ++j)
+                                    v |= (uint32_t)(kb * 4 + j < kg ? __ldg(src + j) : 0x7Fu) << (8 * j);
+                            }
+                        }
+                        w[q] = v;
+                    }
+                    ok = put_stage(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], w[8], w[9], w[10], w[11]);
+                }
             }
         }
-    } else if (warp >= C::FIRST_EPI_WARP) {
+    }
+    } else {
         // ------------------------------------------------ epilogue
+        if (V == V_BLOCK) ptx::regs_inc<224>();
         const int ew = warp - C::FIRST_EPI_WARP;          // 0 .. EPI_WARPS-1
         const int quarter = warp & 3;                      // TMEM lane quarter this warp may access
         const int half = (C::EPI_WARPS == 8) ? (ew >> 2) : 0;   // column half (8-warp variants)
@@ -383,33 +448,66 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 ++acc_it;
             } else if (V == V_BLOCK) {
-                // software promotion over the K blocks
-                float acc[128];
+                // software promotion over the K blocks (pairs of columns, packed FMAs)
+                float2 acc[64];
 #pragma unroll
-                for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+                for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
                 const int32_t nblk = nb * 2 + half;                      // 128-wide weight block
                 const int32_t nbw = (p.N + 127) / 128;
                 const float* sxr = p.sa + (int64_t)(row < p.M ? row : 0) * p.num_kb;
                 const float* swr = p.sb + (int64_t)(nblk < nbw ? nblk : 0) * p.num_kb;
-                float sx_next = __ldg(sxr), sw_next = __ldg(swr);
-                for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-                    const float s = sx_next * sw_next;
-                    if (kb + 1 < p.num_kb) { sx_next = __ldg(sxr + kb + 1); sw_next = __ldg(swr + kb + 1); }
+                // one promotion step: P_kb (in TMEM buffer `buf`) * s added into acc
+                auto promote = [&](float s) -> bool {
                     const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
-                    if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) return false;
                     ptx::tc_fence_after();
+                    const float2 s2 = make_float2(s, s);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        uint32_t r[32];
-                        ptx::tmem_ld_32x32b_x32(tmem_base + lane_base + buf * BN + half * 128 + c * 32, r);
+                        uint32_t r0[16], r1[16];
+                        const uint32_t col = tmem_base + lane_base + buf * BN + half * 128 + c * 32;
+                        ptx::tmem_ld_32x32b_x16(col, r0);
+                        ptx::tmem_ld_32x32b_x16(col + 16, r1);
                         ptx::tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), s, acc[c * 32 + j]);
+                        for (int j = 0; j < 8; ++j) {
+                            acc[c * 16 + j] = ptx::ffma2(
+                                make_float2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), s2,
+                                acc[c * 16 + j]);
+                            acc[c * 16 + 8 + j] = ptx::ffma2(
+                                make_float2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])), s2,
+                                acc[c * 16 + 8 + j]);
+                        }
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
                     ++acc_it;
+                    return true;
+                };
+                if ((p.num_kb & 3) == 0 &&
+                    ((reinterpret_cast<uintptr_t>(p.sa) | reinterpret_cast<uintptr_t>(p.sb)) & 15u) == 0) {
+                    // scales of four K blocks per 16-byte load, fetched one group ahead
+                    float4 cx = __ldg(reinterpret_cast<const float4*>(sxr));
+                    float4 cw = __ldg(reinterpret_cast<const float4*>(swr));
+                    for (int32_t kb = 0; kb < p.num_kb && ok; kb += 4) {
+                        float4 nx = cx, nw = cw;
+                        if (kb + 4 < p.num_kb) {
+                            nx = __ldg(reinterpret_cast<const float4*>(sxr + kb + 4));
+                            nw = __ldg(reinterpret_cast<const float4*>(swr + kb + 4));
+                        }
+                        ok = promote(cx.x * cw.x) && promote(cx.y * cw.y) && promote(cx.z * cw.z) &&
+                             promote(cx.w * cw.w);
+                        cx = nx;
+                        cw = nw;
+                    }
+                } else {
+                    float sx_next = __ldg(sxr), sw_next = __ldg(swr);
+                    for (int32_t kb = 0; kb < p.num_kb && ok; ++kb) {
+                        const float s = sx_next * sw_next;
+                        if (kb + 1 < p.num_kb) { sx_next = __ldg(sxr + kb + 1); sw_next = __ldg(swr + kb + 1); }
+                        ok = promote(s);
+                    }
                 }
                 if (!ok) break;
 #pragma unroll
@@ -417,7 +515,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     const int32_t n0 = nb * BN + half * 128 + c * 32;
                     uint32_t w[16];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) w[j / 2] = pack_bf16x2(acc[c * 32 + j], acc[c * 32 + j + 1]);
+                    for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(acc[c * 16 + j].x, acc[c * 16 + j].y);
                     if (n0 < p.N) {
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
@@ -557,6 +655,19 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
     p.num_kb = (int32_t)((g.K + BK - 1) / BK);
     // keep the operand with the smaller footprint resident in L2: walk its tiles fastest
     p.m_fastest = (g.M <= g.N) ? 1 : 0;
+    {
+        // group the fast dimension so that one group's operand panel is <= ~36 MB
+        const int64_t nfast = p.m_fastest ? p.num_m : p.num_n;
+        const int64_t panel = (int64_t)(p.m_fastest ? BM : BN) * g.K;
+        int64_t grp = std::max<int64_t>(1, (int64_t)36 * 1024 * 1024 / std::max<int64_t>(panel, 1));
+        if (grp >= nfast) {
+            grp = nfast;
+        } else {
+            const int64_t ngroups = (nfast + grp - 1) / grp;
+            grp = (nfast + ngroups - 1) / ngroups;
+        }
+        p.group = (int32_t)std::max<int64_t>(grp, 1);
+    }
     p.status = g.status;
     p.y = g.y;
     p.ldy = g.ldy;
