@@ -461,7 +461,7 @@ def run_quant_sweep(args, torch, fp8, stream, barrier, dist, world, rank, gpu_in
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"],
                          "traffic": profiled_traffic("quant_tensor_quant_sweep"),
-                         "kernel": "amax_partials_kernel + cast_tensor_kernel (one fp8_quantize call)",
+                         "kernel": "rq_amax_kernel + rq_tensor_kernel<CAST> (one fp8_quantize call)",
                          "peak_source": f"{peak_src} hbm_gbs", "call_us_avg": k_ms * 1e3},
             "clocks": clk.summary(), "gpu_launches": args.steps * 4}
     if rank == 0:
@@ -560,7 +560,7 @@ def main():
     variant = {1: "ROWSCALE", 2: "BLOCK", 4: "MX"}[wl["x_mode"]]
     traffic = profiled_traffic(f"gemm_{variant.lower()}_{args.workload}")
     xbytes = M * K * 3 + {1: 4 * M, 2: 4 * M * (-(-K // 128)), 4: M * (K // 32)}[wl["x_mode"]]
-    qkernel = {1: "stream_quant_kernel<ROW>", 2: "stream_quant_kernel<B128>", 4: "stream_quant_kernel<MX>"}[wl["x_mode"]]
+    qkernel = {1: "rq_row_kernel", 2: "rq_block_kernel<B128>", 4: "rq_block_kernel<MX>"}[wl["x_mode"]]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",

@@ -47,6 +47,31 @@ __device__ __forceinline__ float bf16bits_to_float(uint32_t b16) { return __uint
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Lane-wise max of |a|, |b| on packed bf16 pairs; NaN in either input gives NaN
+// (the sign bits of the result are the xor of the inputs' signs: mask them off).
+__device__ __forceinline__ uint32_t bmax_abs_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Packed fp32 pair arithmetic (one instruction for two lanes), round to nearest.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(reinterpret_cast<unsigned long long&>(d))
+        : "l"(reinterpret_cast<const unsigned long long&>(a)), "l"(reinterpret_cast<const unsigned long long&>(b)));
+    return d;
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(reinterpret_cast<unsigned long long&>(d))
+        : "l"(reinterpret_cast<const unsigned long long&>(a)), "l"(reinterpret_cast<const unsigned long long&>(b)),
+          "l"(reinterpret_cast<const unsigned long long&>(c)));
+    return d;
+}
+
 // ---------------------------------------------------------------- FP8 casts
 // Two fp32 values -> two codes (a in the low byte), round-to-nearest-even with
 // saturation to the largest finite value: for finite inputs identical to

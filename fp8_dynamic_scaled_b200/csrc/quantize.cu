@@ -16,7 +16,6 @@
 // patterns (exact and order-free); a pattern >= 0x7F80 flags NaN/Inf input.
 #include "common.cuh"
 #include "kernels.h"
-#include "ptx.cuh"
 
 namespace fp8b {
 
@@ -387,39 +386,123 @@ __global__ void __launch_bounds__(QT) quant_block128_kernel(const uint16_t* __re
     }
 }
 
-// ================================================================ streaming kernels
-// Persistent CTAs stream fixed-size chunks of X through a ring of SQ_NBUF shared-
-// memory buffers filled by 1-D bulk asynchronous copies (one thread issues them,
-// completion on an mbarrier), so SQ_NBUF-1 chunks per CTA are in flight from HBM
-// while the CTA quantises the current chunk out of shared memory.
-//   SQ_AMAX     per-tensor phase 1: running max of |x|, one partial per CTA
-//   SQ_CAST     per-tensor phase 2: s from the partials; chunks are visited in the
-//               reverse of phase 1's order so the most recently read lines of X
-//               (kept with an evict-last L2 policy in phase 1) are reused from L2
-//   SQ_DELAYED  delayed scaling, t >= 1: s from the ring, amax_t reduced on the fly
-//   SQ_ROW      one chunk = one row (per-token / per-channel scale)
-//   SQ_B128     1x128 blocks (16 lanes reduce one block)
-//   SQ_MX       MX32 blocks (4 lanes reduce one block)
-// The division x / s is computed as a reciprocal plus one Markstein correction
-// step: with r = RN(1/s), q = RN(x r), e = RN(x - q s) (exact through the FMA),
+// ================================================================ register-resident kernels
+// The fast path for dense shapes.  Each thread loads all of its 16-byte vectors
+// before using any (VPT or U independent loads in flight), the data stays in
+// registers from the amax through the cast, and small register footprints keep
+// 8 CTAs (2,048 threads) resident per SM, so every SM has >= 128 KB of loads in
+// flight -- enough to cover HBM latency at full bandwidth.  (A design that staged
+// chunks through a shared-memory ring with bulk asynchronous copies was measured
+// slower on B200 for these kernels: 4.9 vs 6.1 TB/s per-token, 4.2 vs 6.1 TB/s for
+// 1x128 blocks.)
+//   RQ_ROW      one CTA per row (per-token / per-channel scale), VPT vectors per thread
+//   RQ_B128     1x128 blocks: 16 consecutive lanes reduce one block
+//   RQ_MX       MX32 blocks: 4 consecutive lanes reduce one block
+//   RQ_AMAX     per-tensor phase 1: grid-stride max of |x|, one partial per CTA
+//   RQ_CAST     per-tensor phase 2: s from the partials, cast in the reverse of
+//               phase 1's order (its last reads are the likeliest L2 hits)
+//   RQ_DELAYED  delayed scaling t >= 1: s from the ring, amax_t reduced on the fly
+//               and committed to the ring by the last CTA to finish
+// The division x / s is a reciprocal plus one Markstein correction step: with
+// r = RN(1/s), q = RN(x r), e = RN(x - q s) (exact through the FMA),
 // RN(q + e r) equals RN(x / s) for every quotient in the fp32 normal range (P.
 // Markstein, "Computation of elementary functions on the IBM RISC System/6000
 // processor", IBM J. Res. Dev. 34(1), 1990).  Quotients below the normal range
 // (|t| < 2^-126) may differ in their last bits, but every such t encodes to a
-// signed zero in both FP8 formats; the sign of x is copied onto t so -0 and tiny
-// negatives keep their sign.
-enum { SQ_AMAX = 0, SQ_CAST = 1, SQ_DELAYED = 2, SQ_ROW = 3, SQ_B128 = 4, SQ_MX = 5 };
-constexpr int SQ_NBUF = 4;
-constexpr int SQ_CHUNK = 8192;              // elements per flat chunk (16 KB of bf16)
-constexpr uint64_t SQ_TIMEOUT_NS = 4000000000ull;
+// signed zero in both FP8 formats.
+enum { RQ_ROW = 0, RQ_B128 = 1, RQ_MX = 2, RQ_AMAX = 3, RQ_CAST = 4, RQ_DELAYED = 5 };
 
-struct SQParams {
+struct RcpScale {
+    float s, r;
+};
+template <int FMT>
+__device__ __forceinline__ RcpScale rcp_scale_from_amax_bits(uint32_t m) {
+    const float s = scale_from_amax<FMT>(bf16bits_to_float(m));
+    return RcpScale{s, __frcp_rn(s)};
+}
+
+// |x| max over the 8 bf16 of a vector with packed bf16 max (the sign bits of the
+// result are meaningless; NaN propagates).
+__device__ __forceinline__ uint32_t vec_amax2_bf(const uint4& v) {
+    return bmax_abs_bf16x2(bmax_abs_bf16x2(v.x, v.y), bmax_abs_bf16x2(v.z, v.w));
+}
+
+// 8 elements -> 8 codes with the Markstein-corrected division on packed pairs.
+// The arithmetic runs on -x with -r: q = RN((-x)(-r)) = RN(x r),
+// e' = RN(q s + (-x)) = -RN(x - q s), t = RN(e' (-r) + q) = RN(q + (x - q s) r);
+// working on -x also makes x = -0 come out as -0 (code 0x80).
+template <int FMT>
+__device__ __forceinline__ uint2 cast_vec_rcp(const uint4& v, const RcpScale& op) {
+    const float2 s2 = make_float2(op.s, op.s);
+    const float2 nr2 = make_float2(-op.r, -op.r);
+    uint32_t c[4];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t wn = w[i] ^ 0x80008000u;
+        const float2 nx = make_float2(__uint_as_float(wn << 16), __uint_as_float(wn & 0xFFFF0000u));
+        const float2 q = mul2_rn(nx, nr2);
+        const float2 e = fma2_rn(q, s2, nx);
+        const float2 t = fma2_rn(e, nr2, q);
+        c[i] = cvt_pair<FMT>(t.x, t.y);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// The same for quotients that may leave the fp32 range (delayed scaling: the
+// history scale can be far below the current amax).  An infinite first quotient
+// saturates to +-F_max as it is and is not corrected (which would give NaN).
+template <int FMT>
+__device__ __forceinline__ uint2 cast_vec_rcp_guarded(const uint4& v, const RcpScale& op) {
+    uint32_t c[4];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float t[2];
+        const float xs[2] = {bf16_lo(w[i]), bf16_hi(w[i])};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float nx = -xs[h];
+            const float q = __fmul_rn(nx, -op.r);
+            const float e = __fmaf_rn(q, op.s, nx);
+            t[h] = fabsf(q) <= 3.402823466e38f ? __fmaf_rn(e, -op.r, q) : q;
+        }
+        c[i] = cvt_pair<FMT>(t[0], t[1]);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// 8 elements -> 8 codes for a power-of-two scale: t = x * 2^-e (exact) on pairs.
+template <int FMT>
+__device__ __forceinline__ uint2 cast_vec_pow2(const uint4& v, float inv) {
+    const float2 i2 = make_float2(inv, inv);
+    uint32_t c[4];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        const float2 t = mul2_rn(x, i2);
+        c[i] = cvt_pair<FMT>(t.x, t.y);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// 8 codes -> 8 bf16 of decode(q) * mul, products on pairs.
+template <int FMT>
+__device__ __forceinline__ uint4 dequant_vec2(const uint2& c, float mul) {
+    const float2 m2 = make_float2(mul, mul);
+    const float2 a = mul2_rn(decode_pair<FMT>(c.x & 0xFFFFu), m2);
+    const float2 b = mul2_rn(decode_pair<FMT>(c.x >> 16), m2);
+    const float2 d = mul2_rn(decode_pair<FMT>(c.y & 0xFFFFu), m2);
+    const float2 e = mul2_rn(decode_pair<FMT>(c.y >> 16), m2);
+    return make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y), pack_bf16x2(d.x, d.y), pack_bf16x2(e.x, e.y));
+}
+
+struct RQParams {
     const uint16_t* x;
-    int64_t ld;           // SQ_ROW: row stride (elements)
-    int64_t n;            // flat kinds: number of elements
-    int64_t cols;         // SQ_ROW: row length
-    int64_t nchunks;
-    int32_t chunk_elems;  // flat kinds: SQ_CHUNK; SQ_ROW: cols
+    int64_t ld;           // RQ_ROW: row stride (elements)
+    int64_t rows, cols;   // RQ_ROW
+    int64_t n;            // flat kinds: number of elements (dense tensor)
     uint8_t* q;
     void* scale;
     uint16_t* deq;
@@ -433,218 +516,164 @@ struct SQParams {
     uint32_t* ticket;
 };
 
-struct RcpScale {
-    float s, r;
-    __device__ __forceinline__ float operator()(float x) const {
-        const float q = __fmul_rn(x, r);
-        const float e = __fmaf_rn(-q, s, x);
-        const float t = __fmaf_rn(e, r, q);
-        return __uint_as_float(__float_as_uint(t) | (__float_as_uint(x) & 0x80000000u));
-    }
-    __device__ __forceinline__ float deq() const { return s; }
-};
-// The same for quotients that may leave the fp32 range (delayed scaling: the
-// history scale can be far below the current amax): an infinite first quotient is
-// kept as is (it saturates to +-F_max), not corrected into a NaN.
-struct RcpScaleGuarded {
-    float s, r;
-    __device__ __forceinline__ float operator()(float x) const {
-        const float q = __fmul_rn(x, r);
-        const float e = __fmaf_rn(-q, s, x);
-        const float t = fabsf(q) <= 3.402823466e38f ? __fmaf_rn(e, r, q) : q;
-        return __uint_as_float(__float_as_uint(t) | (__float_as_uint(x) & 0x80000000u));
-    }
-    __device__ __forceinline__ float deq() const { return s; }
-};
-template <int FMT>
-__device__ __forceinline__ RcpScale rcp_scale_from_amax_bits(uint32_t m) {
-    const float s = scale_from_amax<FMT>(bf16bits_to_float(m));
-    return RcpScale{s, __frcp_rn(s)};
-}
-
-__device__ __forceinline__ bool sq_wait(uint64_t* bar, uint32_t parity) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = ptx::globaltimer();
-    while (!ptx::mbar_try_wait(bar, parity))
-        if (ptx::globaltimer() - t0 > SQ_TIMEOUT_NS) return false;
-    return true;
-}
-
-template <int FMT, bool DEQ, int KIND, int VPT>
-__global__ void __launch_bounds__(QT) stream_quant_kernel(const SQParams p) {
-    extern __shared__ __align__(128) uint8_t sbuf[];
-    __shared__ __align__(8) uint64_t full[SQ_NBUF];
+// One CTA per row; the row (<= QT * VPT vectors) is held in registers.
+template <int FMT, bool DEQ, int VPT, int MINB>
+__global__ void __launch_bounds__(QT, MINB) rq_row_kernel(const RQParams p) {
     __shared__ uint32_t red[32];
-    const int tid = threadIdx.x;
-    const uint32_t buf_bytes = (uint32_t)p.chunk_elems * 2;
-    if (tid == 0) {
-        for (int b = 0; b < SQ_NBUF; ++b) ptx::mbar_init(&full[b], 1);
-        ptx::fence_mbar_init();
+    const int64_t r = blockIdx.x;
+    const uint16_t* src = p.x + r * p.ld;
+    const int64_t nvec = p.cols / VEC;
+    uint4 v[VPT];
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int64_t k = threadIdx.x + (int64_t)QT * j;
+        v[j] = k < nvec ? ld_v4_stream(src + k * VEC) : make_uint4(0, 0, 0, 0);
     }
-    __syncthreads();
-
-    // ---- tensor-wide scale (per-tensor phase 2, delayed)
-    RcpScale op{1.0f, 1.0f};
-    RcpScaleGuarded gop{1.0f, 1.0f};
-    if (KIND == SQ_CAST || KIND == SQ_DELAYED) {
-        uint32_t src = 0;
-        if (KIND == SQ_CAST) {
-            for (int i = tid; i < p.npartials; i += QT) src = max(src, p.partials[i]);
-        } else {
-            for (int i = tid; i < p.ring_len; i += QT) src = max(src, __float_as_uint(p.ring[i]));
-        }
-        src = block_max_u32(src, red);
-        float amax;
-        if (KIND == SQ_CAST) {
-            if (src >= 0x7F80u) {
-                if (blockIdx.x == 0 && tid == 0) report_status(p.status, FP8_ERR_NONFINITE);
-                src = 0x7F7Fu;
-            }
-            amax = bf16bits_to_float(src);
-        } else {
-            amax = __uint_as_float(src);
-        }
-        const float s = scale_from_amax<FMT>(amax);
-        op = RcpScale{s, __frcp_rn(s)};
-        gop = RcpScaleGuarded{s, op.r};
-        if (blockIdx.x == 0 && tid == 0) {
-            reinterpret_cast<float*>(p.scale)[0] = s;
-            if (KIND == SQ_CAST && p.ring != nullptr) p.ring[p.slot] = amax;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(v[j]));
+    uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
+    if (m >= 0x7F80u) {
+        if (threadIdx.x == 0) report_status(p.status, FP8_ERR_NONFINITE);
+        m = 0x7F7Fu;
+    }
+    const RcpScale op = rcp_scale_from_amax_bits<FMT>(m);
+    if (threadIdx.x == 0) reinterpret_cast<float*>(p.scale)[r] = op.s;
+    uint8_t* dst = p.q + r * p.cols;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int64_t k = threadIdx.x + (int64_t)QT * j;
+        if (k < nvec) {
+            const uint2 cq = cast_vec_rcp<FMT>(v[j], op);
+            *reinterpret_cast<uint2*>(dst + k * VEC) = cq;
+            if (DEQ) st_v4_stream(p.deq + r * p.cols + k * VEC, dequant_vec2<FMT>(cq, op.s));
         }
     }
+}
 
-    const int64_t first = blockIdx.x;
-    const int64_t n_mine = first < p.nchunks ? (p.nchunks - 1 - first) / gridDim.x + 1 : 0;
-    const uint64_t policy = KIND == SQ_AMAX ? ptx::l2_policy_evict_last() : ptx::l2_policy_evict_first();
-    auto chunk_id = [&](int64_t i) -> int64_t {
-        const int64_t c = first + i * (int64_t)gridDim.x;
-        return KIND == SQ_CAST ? p.nchunks - 1 - c : c;
+// 1x128 / MX32 blocks of a dense tensor: each CTA takes QT * VPT consecutive vectors;
+// for a fixed j the vectors of one block sit in G consecutive lanes.
+template <int FMT, bool DEQ, int KIND, int VPT>
+__global__ void __launch_bounds__(QT, 8) rq_block_kernel(const RQParams p) {
+    constexpr int G = KIND == RQ_B128 ? 16 : 4;
+    const int64_t e0 = (int64_t)blockIdx.x * QT * VPT * VEC;
+    uint4 v[VPT];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int64_t off = e0 + (int64_t)(threadIdx.x + QT * j) * VEC;
+        v[j] = off < p.n ? ld_v4_stream(p.x + off) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        uint32_t m = hmax_pair(vec_amax2_bf(v[j]) & 0x7FFF7FFFu);
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const int vec = threadIdx.x + QT * j;
+        const int64_t off = e0 + (int64_t)vec * VEC;
+        if (off >= p.n) continue;
+        if (m >= 0x7F80u) {
+            report_status(p.status, FP8_ERR_NONFINITE);
+            m = 0x7F7Fu;
+        }
+        uint2 cq;
+        float dmul;
+        if (KIND == RQ_B128) {
+            const RcpScale op = rcp_scale_from_amax_bits<FMT>(m);
+            if ((vec & (G - 1)) == 0) reinterpret_cast<float*>(p.scale)[off / 128] = op.s;
+            cq = cast_vec_rcp<FMT>(v[j], op);
+            dmul = op.s;
+        } else {
+            const int e = mx_exponent(m);
+            if ((vec & (G - 1)) == 0) reinterpret_cast<uint8_t*>(p.scale)[off / 32] = (uint8_t)(e + 127);
+            cq = cast_vec_pow2<FMT>(v[j], exp2i(-e));
+            dmul = exp2i(e);
+        }
+        *reinterpret_cast<uint2*>(p.q + off) = cq;
+        if (DEQ) st_v4_stream(p.deq + off, dequant_vec2<FMT>(cq, dmul));
+    }
+}
+
+// Per-tensor phase 1: U independent loads in flight per thread.
+template <int U>
+__global__ void __launch_bounds__(QT, 8) rq_amax_kernel(const RQParams p) {
+    __shared__ uint32_t red[32];
+    const int64_t nvec = p.n / VEC;
+    uint32_t m2 = 0;
+    const int64_t stride = (int64_t)gridDim.x * QT;
+    int64_t v = (int64_t)blockIdx.x * QT + threadIdx.x;
+    for (; v + (U - 1) * stride < nvec; v += U * stride) {
+        uint4 a[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) a[u] = ld_v4(p.x + (v + u * stride) * VEC);
+#pragma unroll
+        for (int u = 0; u < U; ++u) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(a[u]));
+    }
+    for (; v < nvec; v += stride) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(ld_v4(p.x + v * VEC)));
+    const uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
+    if (threadIdx.x == 0) p.partials[blockIdx.x] = m;
+}
+
+// Per-tensor phase 2 (RQ_CAST) or the delayed single pass (RQ_DELAYED).
+template <int FMT, bool DEQ, int KIND, int U>
+__global__ void __launch_bounds__(QT, 6) rq_tensor_kernel(const RQParams p) {
+    __shared__ uint32_t red[32];
+    uint32_t src = 0;
+    if (KIND == RQ_CAST) {
+        for (int i = threadIdx.x; i < p.npartials; i += QT) src = max(src, p.partials[i]);
+    } else {
+        for (int i = threadIdx.x; i < p.ring_len; i += QT) src = max(src, __float_as_uint(p.ring[i]));
+    }
+    src = block_max_u32(src, red);
+    float amax;
+    if (KIND == RQ_CAST) {
+        if (src >= 0x7F80u) {
+            if (blockIdx.x == 0 && threadIdx.x == 0) report_status(p.status, FP8_ERR_NONFINITE);
+            src = 0x7F7Fu;
+        }
+        amax = bf16bits_to_float(src);
+    } else {
+        amax = __uint_as_float(src);
+    }
+    const float s = scale_from_amax<FMT>(amax);
+    const RcpScale op{s, __frcp_rn(s)};
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        reinterpret_cast<float*>(p.scale)[0] = s;
+        if (KIND == RQ_CAST && p.ring != nullptr) p.ring[p.slot] = amax;
+    }
+    const int64_t nvec = p.n / VEC;
+    const int64_t stride = (int64_t)gridDim.x * QT;
+    uint32_t m2 = 0;
+    auto vec_of = [&](int64_t t) -> int64_t { return KIND == RQ_CAST ? nvec - 1 - t : t; };
+    auto emit = [&](int64_t vv, const uint4& a) {
+        uint2 cq;
+        if (KIND == RQ_DELAYED) {
+            m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(a));
+            cq = cast_vec_rcp_guarded<FMT>(a, op);
+        } else {
+            cq = cast_vec_rcp<FMT>(a, op);
+        }
+        *reinterpret_cast<uint2*>(p.q + vv * VEC) = cq;
+        if (DEQ) st_v4_stream(p.deq + vv * VEC, dequant_vec2<FMT>(cq, s));
     };
-    auto issue = [&](int64_t i) {
-        const int64_t c = chunk_id(i);
-        const int b = (int)(i % SQ_NBUF);
-        const uint16_t* src;
-        uint32_t bytes;
-        if (KIND == SQ_ROW) {
-            src = p.x + c * p.ld;
-            bytes = (uint32_t)(p.cols * 2);
-        } else {
-            const int64_t e0 = c * p.chunk_elems;
-            const int64_t ne = min((int64_t)p.chunk_elems, p.n - e0);
-            src = p.x + e0;
-            bytes = (uint32_t)(ne * 2);
-        }
-        ptx::mbar_arrive_expect_tx(&full[b], bytes);
-        ptx::bulk_load_1d(sbuf + (size_t)b * buf_bytes, src, bytes, &full[b], policy);
-    };
-    if (tid == 0)
-        for (int64_t i = 0; i < n_mine && i < SQ_NBUF; ++i) issue(i);
-
-    uint32_t m2_run = 0;   // running |x| max (SQ_AMAX, SQ_DELAYED), packed pair
-    for (int64_t i = 0; i < n_mine; ++i) {
-        const int b = (int)(i % SQ_NBUF);
-        const bool ok = sq_wait(&full[b], (uint32_t)((i / SQ_NBUF) & 1));
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) report_status(p.status, FP8_ERR_TIMEOUT);
-            break;
-        }
-        const int64_t c = chunk_id(i);
-        const uint8_t* buf = sbuf + (size_t)b * buf_bytes;
-        const int64_t e0 = KIND == SQ_ROW ? c * p.cols : c * (int64_t)p.chunk_elems;
-        const int64_t ne = KIND == SQ_ROW ? p.cols : min((int64_t)p.chunk_elems, p.n - e0);
-        uint4 v[VPT];
-        bool has[VPT];
+    int64_t t = (int64_t)blockIdx.x * QT + threadIdx.x;
+    for (; t + (U - 1) * stride < nvec; t += U * stride) {
+        uint4 a[U];
 #pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-            const int vec = tid + QT * j;
-            has[j] = (int64_t)vec * VEC < ne;
-            v[j] = has[j] ? *reinterpret_cast<const uint4*>(buf + (size_t)vec * 16) : make_uint4(0, 0, 0, 0);
-        }
-        if (KIND == SQ_AMAX) {
+        for (int u = 0; u < U; ++u) a[u] = ld_v4(p.x + vec_of(t + u * stride) * VEC);
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) m2_run = max_bf16x2_bits(m2_run, vec_amax2(v[j]));
-        } else if (KIND == SQ_CAST || KIND == SQ_DELAYED) {
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                if (!has[j]) continue;
-                const int64_t off = e0 + (int64_t)(tid + QT * j) * VEC;
-                uint2 cq;
-                if (KIND == SQ_DELAYED) {
-                    m2_run = max_bf16x2_bits(m2_run, vec_amax2(v[j]));
-                    cq = cast_vec<FMT>(v[j], gop);
-                } else {
-                    cq = cast_vec<FMT>(v[j], op);
-                }
-                *reinterpret_cast<uint2*>(p.q + off) = cq;
-                if (DEQ) st_v4_stream(p.deq + off, dequant_vec<FMT>(cq, op.s));
-            }
-        } else if (KIND == SQ_ROW) {
-            uint32_t m2 = 0;
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) m2 = max_bf16x2_bits(m2, vec_amax2(v[j]));
-            uint32_t m = block_max_u32(hmax_pair(m2), red);
-            if (m >= 0x7F80u) {
-                if (tid == 0) report_status(p.status, FP8_ERR_NONFINITE);
-                m = 0x7F7Fu;
-            }
-            const RcpScale rop = rcp_scale_from_amax_bits<FMT>(m);
-            if (tid == 0) reinterpret_cast<float*>(p.scale)[c] = rop.s;
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                if (!has[j]) continue;
-                const int64_t off = e0 + (int64_t)(tid + QT * j) * VEC;
-                const uint2 cq = cast_vec<FMT>(v[j], rop);
-                *reinterpret_cast<uint2*>(p.q + off) = cq;
-                if (DEQ) st_v4_stream(p.deq + off, dequant_vec<FMT>(cq, rop.s));
-            }
-        } else {   // SQ_B128 / SQ_MX: groups of G consecutive lanes own one block
-            constexpr int G = KIND == SQ_B128 ? 16 : 4;
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                uint32_t m = hmax_pair(vec_amax2(v[j]));
-#pragma unroll
-                for (int o = G / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (!has[j]) continue;
-                if (m >= 0x7F80u) {
-                    report_status(p.status, FP8_ERR_NONFINITE);
-                    m = 0x7F7Fu;
-                }
-                const int vec = tid + QT * j;
-                const int64_t off = e0 + (int64_t)vec * VEC;
-                uint2 cq;
-                float dmul;
-                if (KIND == SQ_B128) {
-                    const RcpScale rop = rcp_scale_from_amax_bits<FMT>(m);
-                    if ((vec & (G - 1)) == 0) reinterpret_cast<float*>(p.scale)[off / 128] = rop.s;
-                    cq = cast_vec<FMT>(v[j], rop);
-                    dmul = rop.s;
-                } else {
-                    const int e = mx_exponent(m);
-                    const Pow2Scale pop{exp2i(-e), exp2i(e)};
-                    if ((vec & (G - 1)) == 0) reinterpret_cast<uint8_t*>(p.scale)[off / 32] = (uint8_t)(e + 127);
-                    cq = cast_vec<FMT>(v[j], pop);
-                    dmul = pop.mul;
-                }
-                *reinterpret_cast<uint2*>(p.q + off) = cq;
-                if (DEQ) st_v4_stream(p.deq + off, dequant_vec<FMT>(cq, dmul));
-            }
-        }
-        __syncthreads();   // every thread is done with buffer b
-        if (tid == 0 && i + SQ_NBUF < n_mine) issue(i + SQ_NBUF);
+        for (int u = 0; u < U; ++u) emit(vec_of(t + u * stride), a[u]);
     }
-
-    if (KIND == SQ_AMAX) {
-        const uint32_t m = block_max_u32(hmax_pair(m2_run), red);
-        if (tid == 0) p.partials[blockIdx.x] = m;
-    }
-    if (KIND == SQ_DELAYED) {
-        const uint32_t m = block_max_u32(hmax_pair(m2_run), red);
-        if (tid == 0) {
+    for (; t < nvec; t += stride) emit(vec_of(t), ld_v4(p.x + vec_of(t) * VEC));
+    if (KIND == RQ_DELAYED) {
+        const uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
+        if (threadIdx.x == 0) {
             if (m >= 0x7F80u) report_status(p.status, FP8_ERR_NONFINITE);
+            // amax >= 0, so the fp32 bit pattern orders like the value
             atomicMax(reinterpret_cast<uint32_t*>(p.pending), m << 16);
             __threadfence();
-            const uint32_t t = atomicAdd(p.ticket, 1u);
-            if (t == gridDim.x - 1) {
+            const uint32_t ticket = atomicAdd(p.ticket, 1u);
+            if (ticket == gridDim.x - 1) {
+                // every CTA read the ring before taking its ticket
                 __threadfence();
                 const uint32_t a_t = atomicOr(reinterpret_cast<uint32_t*>(p.pending), 0u);
                 p.ring[p.slot] = __uint_as_float(a_t);
@@ -692,62 +721,41 @@ static void launch_cast_tensor(const QuantArgs& a, int src, dim3 grid, int npart
             (float*)a.scale, a.deq, a.status);
 }
 
-// Persistent grid for a streaming kernel: as many CTAs as fit on the GPU at this
-// shared-memory size (at most amax_partials_count(), the per-tensor workspace size).
-template <int FMT, bool DEQ, int KIND, int VPT>
-static cudaError_t launch_sq(const SQParams& p, cudaStream_t st, int* grid_out = nullptr) {
-    auto kern = stream_quant_kernel<FMT, DEQ, KIND, VPT>;
-    const int smem = SQ_NBUF * p.chunk_elems * 2;
-    static int attr_set = 0;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SQ_NBUF * 16384 * 2);
-        if (e != cudaSuccess) return e;
-        attr_set = 1;
-    }
-    int occ = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, QT, smem);
-    if (e != cudaSuccess) return e;
-    occ = std::max(occ, 1);
-    const int64_t grid = std::max<int64_t>(
-        1, std::min<int64_t>({p.nchunks, (int64_t)occ * sm_count_cached(), (int64_t)amax_partials_count()}));
-    if (grid_out) *grid_out = (int)grid;
-    kern<<<(unsigned)grid, QT, smem, st>>>(p);
-    return cudaGetLastError();
-}
+static int64_t rq_grid_cap() { return std::min<int64_t>(amax_partials_count(), (int64_t)sm_count_cached() * 8); }
 
 template <int FMT, bool DEQ>
-static cudaError_t stream_tensor_t(const QuantArgs& a, cudaStream_t st) {
-    SQParams p{};
+static cudaError_t rq_tensor_t(const QuantArgs& a, cudaStream_t st) {
+    RQParams p{};
     p.x = a.x;
-    p.ld = a.ld;
     p.n = a.rows * a.cols;
-    p.nchunks = (p.n + SQ_CHUNK - 1) / SQ_CHUNK;
-    p.chunk_elems = SQ_CHUNK;
     p.q = a.q;
     p.scale = a.scale;
     p.deq = a.deq;
     p.status = a.status;
     p.partials = a.partials;
-    const bool delayed_t = a.hist_ring != nullptr && a.hist_step > 0;
     p.ring = a.hist_ring;
     p.ring_len = a.hist_len;
     p.slot = a.hist_ring ? (int32_t)(a.hist_step % a.hist_len) : 0;
     p.pending = a.hist_pending;
     p.ticket = a.hist_ticket;
-    if (delayed_t) return launch_sq<FMT, DEQ, SQ_DELAYED, 4>(p, st);
-    int grid = 0;
-    cudaError_t e = launch_sq<FMT, false, SQ_AMAX, 4>(p, st, &grid);
-    if (e != cudaSuccess) return e;
-    p.npartials = grid;
-    return launch_sq<FMT, DEQ, SQ_CAST, 4>(p, st);
+    const int64_t nvec = p.n / VEC;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rq_grid_cap(), (nvec + QT - 1) / QT));
+    if (a.hist_ring != nullptr && a.hist_step > 0) {
+        rq_tensor_kernel<FMT, DEQ, RQ_DELAYED, 4><<<(unsigned)grid, QT, 0, st>>>(p);
+        return cudaGetLastError();
+    }
+    rq_amax_kernel<8><<<(unsigned)grid, QT, 0, st>>>(p);
+    p.npartials = (int32_t)grid;
+    rq_tensor_kernel<FMT, DEQ, RQ_CAST, 4><<<(unsigned)grid, QT, 0, st>>>(p);
+    return cudaGetLastError();
 }
 
 // Per-tensor current scaling (two launches) or one delayed step.
 cudaError_t launch_quantize_tensor(const QuantArgs& a, cudaStream_t st) {
     const bool dense = a.ld == a.cols;
     if (dense && a.rows > 0 && a.cols > 0) {
-        if (a.fmt == FP8_E4M3) return a.deq ? stream_tensor_t<FP8_E4M3, true>(a, st) : stream_tensor_t<FP8_E4M3, false>(a, st);
-        return a.deq ? stream_tensor_t<FP8_E5M2, true>(a, st) : stream_tensor_t<FP8_E5M2, false>(a, st);
+        if (a.fmt == FP8_E4M3) return a.deq ? rq_tensor_t<FP8_E4M3, true>(a, st) : rq_tensor_t<FP8_E4M3, false>(a, st);
+        return a.deq ? rq_tensor_t<FP8_E5M2, true>(a, st) : rq_tensor_t<FP8_E5M2, false>(a, st);
     }
     const int64_t nrows = dense ? (a.rows > 0 ? 1 : 0) : a.rows;
     const int64_t nvec = dense ? a.rows * a.cols / VEC : a.cols / VEC;
@@ -789,33 +797,37 @@ static void launch_segment(const QuantArgs& a, int32_t seg_vec, cudaStream_t st)
 
 template <int FMT, bool DEQ>
 static cudaError_t quantize_grouped_t(const QuantArgs& a, cudaStream_t st) {
-    // streaming kernels for the shapes they cover (rows of 1-16 Ki elements; dense
-    // tensors for the 1x128 and MX32 blocks)
+    // register-resident kernels for the shapes they cover (rows of 1-16 Ki elements;
+    // dense tensors for the 1x128 and MX32 blocks)
     {
-        SQParams p{};
+        RQParams p{};
         p.x = a.x;
         p.ld = a.ld;
+        p.rows = a.rows;
+        p.cols = a.cols;
+        p.n = a.rows * a.cols;
         p.q = a.q;
         p.scale = a.scale;
         p.deq = a.deq;
         p.status = a.status;
-        if (a.mode == FP8_SCALE_ROW && a.cols >= 1024 && a.cols <= 16384 && a.rows > 0) {
-            p.cols = a.cols;
-            p.nchunks = a.rows;
-            p.chunk_elems = (int32_t)a.cols;
+        if (a.mode == FP8_SCALE_ROW && a.cols >= 1024 && a.cols <= 16384 && a.rows > 0 && a.rows < ((int64_t)1 << 31)) {
+            const unsigned g = (unsigned)a.rows;
             const int64_t vpt = (a.cols / VEC + QT - 1) / QT;
-            if (vpt <= 1) return launch_sq<FMT, DEQ, SQ_ROW, 1>(p, st);
-            if (vpt <= 2) return launch_sq<FMT, DEQ, SQ_ROW, 2>(p, st);
-            if (vpt <= 4) return launch_sq<FMT, DEQ, SQ_ROW, 4>(p, st);
-            return launch_sq<FMT, DEQ, SQ_ROW, 8>(p, st);
+            if (vpt <= 1)      rq_row_kernel<FMT, DEQ, 1, 8><<<g, QT, 0, st>>>(p);
+            else if (vpt <= 2) rq_row_kernel<FMT, DEQ, 2, 8><<<g, QT, 0, st>>>(p);
+            else if (vpt <= 4) rq_row_kernel<FMT, DEQ, 4, 8><<<g, QT, 0, st>>>(p);
+            else               rq_row_kernel<FMT, DEQ, 8, 4><<<g, QT, 0, st>>>(p);
+            return cudaGetLastError();
         }
         const bool dense = a.ld == a.cols && a.rows > 0 && a.cols > 0;
         if (dense && ((a.mode == FP8_SCALE_BLOCK_1x128 && a.cols % 128 == 0) || a.mode == FP8_SCALE_MX32)) {
-            p.n = a.rows * a.cols;
-            p.nchunks = (p.n + SQ_CHUNK - 1) / SQ_CHUNK;
-            p.chunk_elems = SQ_CHUNK;
-            if (a.mode == FP8_SCALE_MX32) return launch_sq<FMT, DEQ, SQ_MX, 4>(p, st);
-            return launch_sq<FMT, DEQ, SQ_B128, 4>(p, st);
+            const int64_t per_cta = (int64_t)QT * 4 * VEC;
+            const int64_t grid = (p.n + per_cta - 1) / per_cta;
+            if (grid < ((int64_t)1 << 31)) {
+                if (a.mode == FP8_SCALE_MX32) rq_block_kernel<FMT, DEQ, RQ_MX, 4><<<(unsigned)grid, QT, 0, st>>>(p);
+                else                          rq_block_kernel<FMT, DEQ, RQ_B128, 4><<<(unsigned)grid, QT, 0, st>>>(p);
+                return cudaGetLastError();
+            }
         }
     }
     switch (a.mode) {
