@@ -573,7 +573,7 @@ def main():
                          f"{N * K / 1e6:.0f} MB W codes, writes {2 * M * N / 1e6:.0f} MB Y)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": sustained, "unit": "TFLOP/s",
                      "frac": gemm_tflops / sustained, "traffic": traffic,
-                     "kernel": f"fp8_gemm_kernel<{variant}>",
+                     "kernel": "fp8_gemm_pair_kernel" if variant == "ROWSCALE" and M >= 256 else f"fp8_gemm_kernel<{variant}>",
                      "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16} (fp8/bf16 nominal ratio)",
                      "gemm_us_avg": g_avg * 1e3},
         "quantize": {"kernel": qkernel, "us_avg": q_avg * 1e3, "algorithmic_bytes": xbytes,

@@ -564,6 +564,211 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if (warp == 1) ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
+// ================================================================ CTA-pair kernel
+// Per-tensor / per-row scales with tcgen05.mma.cta_group::2: a cluster of two CTAs
+// (one per SM) owns a 256 x 256 output tile.  Each CTA loads its own 128 rows of A
+// and its own 128 rows of B (no multicast), so each SM streams 8 KB of operands per
+// 128-cycle MMA instead of 12 KB; the leader CTA issues M=256 N=256 K=32 MMAs that
+// read both CTAs' shared memory and accumulate 128 rows into each CTA's TMEM.
+//   warp 0   TMA producer (both CTAs), completion on the local full[] barrier
+//   warp 1   TMEM allocator (both CTAs, cta_group::2); MMA issuer (leader only)
+//   warp 2   relay (both CTAs): local full[] -> one arrival on the leader's ready[]
+//   warps 3-6 epilogue (both CTAs) on the CTA's own 128 accumulator rows; they
+//            release an accumulator with one arrival each on the leader's tempty[]
+// The leader's commits arrive on empty[] / tfull[] in both CTAs (multicast commit).
+constexpr int P_BM = 256;                                  // rows per CTA-pair tile
+constexpr int P_STAGES = 6;
+constexpr uint32_t P_HALF_BYTES = 128 * BK;                // 16 KB: one CTA's half of A or B
+struct PairSmem {
+    static constexpr int NT = 7 * 32;
+    static constexpr int EPI_WARPS = 4, FIRST_EPI_WARP = 3, STAGE_BUFS = 2;
+    static constexpr uint32_t A_OFF = 0;
+    static constexpr uint32_t B_OFF = A_OFF + P_STAGES * P_HALF_BYTES;
+    static constexpr uint32_t Y_OFF = B_OFF + P_STAGES * P_HALF_BYTES;
+    static constexpr uint32_t Y_BYTES = EPI_WARPS * STAGE_BUFS * 2048;
+    static constexpr uint32_t BAR_OFF = Y_OFF + Y_BYTES;
+    // full[S], ready[S], empty[S], tfull[2], tempty[2], teardown
+    static constexpr uint32_t BAR_BYTES = 8 * (3 * P_STAGES + 5);
+    static constexpr uint32_t MISC_OFF = BAR_OFF + BAR_BYTES;
+    static constexpr uint32_t TOTAL = MISC_OFF + 16;
+    static constexpr uint32_t ALLOC = TOTAL + 1024;
+};
+
+__global__ void __launch_bounds__(PairSmem::NT, 1)
+fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+    using S = PairSmem;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem + S::A_OFF;
+    uint8_t* sB = smem + S::B_OFF;
+    uint8_t* sY = smem + S::Y_OFF;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+    uint64_t* ready = full + P_STAGES;
+    uint64_t* empty = ready + P_STAGES;
+    uint64_t* tfull = empty + P_STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* teardown = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::MISC_OFF);
+    volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + S::MISC_OFF + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = rank == 0;
+    const int32_t cluster = blockIdx.x >> 1;
+    const int32_t nclusters = gridDim.x >> 1;
+    const int32_t num_tiles = p.num_m * p.num_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&ready[s], 2);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], 2 * S::EPI_WARPS);
+        }
+        ptx::mbar_init(teardown, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        if (!p.y_direct) ptx::prefetch_tmap(&tmY);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(tmem_slot, 512);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
+                int32_t mb, nb;
+                tile_coords(p, t, mb, nb);
+                for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&full[stage], 2 * P_HALF_BYTES);
+                    ptx::tma_load_2d(sA + stage * P_HALF_BYTES, &tmA, &full[stage], kb * BK, mb * P_BM + (int32_t)rank * 128);
+                    ptx::tma_load_2d(sB + stage * P_HALF_BYTES, &tmB, &full[stage], kb * BK, nb * BN + (int32_t)rank * 128);
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------ relay (both CTAs)
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
+                for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                    ptx::mbar_arrive_cluster(&ready[stage], 0);
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (leader) {
+            uint32_t stage = 0, phase = 0, acc_it = 0;
+            bool ok = true;
+            const uint32_t sA0 = ptx::smem_u32(sA), sB0 = ptx::smem_u32(sB);
+            for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
+                const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
+                if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(&ready[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int k = 0; k < BK / UMMA_K; ++k) {
+                            const uint64_t ad = ptx::sdesc_kmajor_sw128(sA0 + stage * P_HALF_BYTES + k * UMMA_K);
+                            const uint64_t bd = ptx::sdesc_kmajor_sw128(sB0 + stage * P_HALF_BYTES + k * UMMA_K);
+                            ptx::mma_f8f6f4_pair(tmem_base + buf * BN, ad, bd, p.idesc, (kb | k) != 0);
+                        }
+                        ptx::mma_commit_pair(&empty[stage], 0x3);
+                    }
+                    __syncwarp();
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                if (lane == 0) ptx::mma_commit_pair(&tfull[buf], 0x3);
+                __syncwarp();
+                ++acc_it;
+            }
+            if (lane == 0) {
+                ptx::mma_commit_pair(teardown, 0x1);
+                wait_bounded(teardown, 0, abort_flag, p.status);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - S::FIRST_EPI_WARP;
+        const int quarter = warp & 3;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        uint8_t* ybuf = sY + ew * S::STAGE_BUFS * 2048;
+        uint32_t acc_it = 0, store_it = 0;
+        bool ok = true;
+        for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
+            int32_t mb, nb;
+            tile_coords(p, t, mb, nb);
+            const int32_t y_row0 = mb * P_BM + (int32_t)rank * 128 + quarter * 32;
+            const int32_t row = y_row0 + lane;
+            const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
+            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const float sx = row < p.M ? __ldg(p.sa + (int64_t)row * p.sa_stride) : 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                ptx::tmem_ld_32x32b_x32(tmem_base + lane_base + buf * BN + c * 32, r);
+                ptx::tmem_ld_wait();
+                if (c == BN / 32 - 1) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive_cluster(&tempty[buf], 0);
+                }
+                const int32_t n0 = nb * BN + c * 32;
+                uint32_t w[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const int32_t n = n0 + j;
+                    const float s0 = n < p.N ? sx * __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
+                    const float s1 = n + 1 < p.N ? sx * __ldg(p.sb + (int64_t)(n + 1) * p.sb_stride) : 0.0f;
+                    w[j / 2] = pack_bf16x2(__uint_as_float(r[j]) * s0, __uint_as_float(r[j + 1]) * s1);
+                }
+                if (n0 < p.N) {
+                    uint8_t* b = ybuf + (store_it % S::STAGE_BUFS) * 2048;
+                    if (lane == 0) ptx::bulk_wait_read<S::STAGE_BUFS - 1>();
+                    __syncwarp();
+                    store_chunk(&tmY, b, w, n0, y_row0, lane, p);
+                    ++store_it;
+                }
+            }
+            ++acc_it;
+        }
+        if (lane == 0) ptx::bulk_wait_all();
+        __syncwarp();
+    }
+
+    // ------------------------------------------------ teardown (both CTAs)
+    ptx::tc_fence_before();
+    ptx::cluster_sync();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc_pair(tmem_base, 512);
+}
+
 // ================================================================ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -632,6 +837,70 @@ static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaSt
     return cudaGetLastError();
 }
 
+// Raster group for a given row-tile height (see tile_coords).
+static int32_t raster_group(int64_t nfast, int64_t panel_bytes) {
+    int64_t grp = std::max<int64_t>(1, (int64_t)36 * 1024 * 1024 / std::max<int64_t>(panel_bytes, 1));
+    if (grp >= nfast) return (int32_t)std::max<int64_t>(nfast, 1);
+    const int64_t ngroups = (nfast + grp - 1) / grp;
+    return (int32_t)std::max<int64_t>((nfast + ngroups - 1) / ngroups, 1);
+}
+
+// CTA-pair launch: clusters of two CTAs, 256 x 256 tiles.
+static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st) {
+    p.num_m = (int32_t)((g.M + P_BM - 1) / P_BM);
+    p.m_fastest = (g.M <= g.N) ? 1 : 0;
+    p.group = raster_group(p.m_fastest ? p.num_m : p.num_n, (int64_t)(p.m_fastest ? P_BM : BN) * g.K);
+    p.idesc = (p.idesc & ~(0x1Fu << 24)) | ((uint32_t)(P_BM >> 4) << 24);
+    CUtensorMap ta, tb, ty;
+    if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.K, BK, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    memset(&ty, 0, sizeof(ty));
+    if (!p.y_direct && !make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, (uint64_t)g.N, (uint64_t)g.M,
+                                    (uint64_t)g.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    static int max_clusters = 0;
+    if (max_clusters == 0) {
+        cudaError_t e = cudaFuncSetAttribute(fp8_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)PairSmem::ALLOC);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(2 * (num_sms() / 2));
+        q.blockDim = dim3(PairSmem::NT);
+        q.dynamicSmemBytes = PairSmem::ALLOC;
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = 2;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        q.attrs = qa;
+        q.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_pair_kernel, &q);
+        if (e != cudaSuccess || n <= 0) n = num_sms() / 2;
+        max_clusters = n;
+    }
+    const int32_t tiles = p.num_m * p.num_n;
+    const int clusters = std::max(1, std::min(tiles, max_clusters));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(PairSmem::NT);
+    cfg.dynamicSmemBytes = PairSmem::ALLOC;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_pair_kernel, ta, tb, ty, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 // Instruction descriptor, kind::f8f6f4: D = F32 (bits 4-5 = 1), A/B formats in bits
 // 7-9 / 10-12 (E4M3 = 0, E5M2 = 1), both K-major, N>>3 in bits 17-22, M>>4 in 24-28.
 static uint32_t idesc_f8f6f4(int fa, int fb) {
@@ -655,19 +924,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
     p.num_kb = (int32_t)((g.K + BK - 1) / BK);
     // keep the operand with the smaller footprint resident in L2: walk its tiles fastest
     p.m_fastest = (g.M <= g.N) ? 1 : 0;
-    {
-        // group the fast dimension so that one group's operand panel is <= ~36 MB
-        const int64_t nfast = p.m_fastest ? p.num_m : p.num_n;
-        const int64_t panel = (int64_t)(p.m_fastest ? BM : BN) * g.K;
-        int64_t grp = std::max<int64_t>(1, (int64_t)36 * 1024 * 1024 / std::max<int64_t>(panel, 1));
-        if (grp >= nfast) {
-            grp = nfast;
-        } else {
-            const int64_t ngroups = (nfast + grp - 1) / grp;
-            grp = (nfast + ngroups - 1) / ngroups;
-        }
-        p.group = (int32_t)std::max<int64_t>(grp, 1);
-    }
+    // group the fast dimension so that one group's operand panel is <= ~36 MB
+    p.group = raster_group(p.m_fastest ? p.num_m : p.num_n, (int64_t)(p.m_fastest ? BM : BN) * g.K);
     p.status = g.status;
     p.y = g.y;
     p.ldy = g.ldy;
@@ -680,6 +938,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
         p.sa_stride = a_pt ? 0 : 1;
         p.sb_stride = b_pt ? 0 : 1;
         p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
+        // CTA pairs once M spans a 256-row tile; a single CTA per tile below that
+        if (g.M >= P_BM) return launch_pair(g, p, st);
         return launch_variant<V_ROWSCALE>(g, p, st);
     }
     if (g.a_mode == FP8_SCALE_BLOCK_1x128 && g.b_mode == FP8_SCALE_BLOCK_128x128) {
