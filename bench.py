@@ -45,6 +45,26 @@ WORKLOADS = {
 }
 
 
+def max_over_ranks(value_ms: float, dist=None, device="cpu") -> float:
+    """The job's time is the slowest rank's (device-timed) time."""
+    if dist is None:
+        return value_ms
+    import torch
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Aggregate throughput of `world` ranks that each processed `units_per_rank` in `ms`."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
+def rank_batch(x: np.ndarray, rank: int) -> np.ndarray:
+    """Each rank's own batch (weak scaling): the seeded batch, rows rotated by rank."""
+    return np.roll(x, rank, axis=0) if rank else x
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -143,8 +163,7 @@ def make_workload(torch, fp8, name, rank):
         x, w = inputs.block_scaled(M, K, N)
     else:
         x, w = inputs.mx_delayed(M, K, N)
-    if rank:
-        x = np.roll(x, rank, axis=0)
+    x = rank_batch(x, rank)
     xd = to_dev_bf16(torch, x)
     wd = to_dev_bf16(torch, w)
     wq, ws, _ = fp8.empty_quant_outputs(N, K, wl["w_mode"])
@@ -403,9 +422,7 @@ def run_quant_sweep(args, torch, fp8, stream, barrier, dist, world, rank, gpu_in
     [1e-6, 1e4], random signs, 1e-4 outliers at +-1e5); one step = per-tensor current
     scaling to E4M3 and to E5M2, each emitting codes + fp32 scale + dequantised bf16."""
     from fp8_dynamic_scaled_b200 import inputs
-    xh = inputs.quant_sweep()
-    if rank:
-        xh = np.roll(xh, rank, axis=0)
+    xh = rank_batch(inputs.quant_sweep(), rank)
     x = to_dev_bf16(torch, xh)
     rows, cols = x.shape
     T = fp8.FP8_SCALE_TENSOR
@@ -443,13 +460,9 @@ def run_quant_sweep(args, torch, fp8, stream, barrier, dist, world, rank, gpu_in
         barrier()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())}")
-    total_ms = start.elapsed_time(end)
-    if dist:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), dist, "cuda")
     ms = total_ms / args.steps
-    value = world * 2 * per_fmt / (ms * 1e-3) / 1e9
+    value = whole_job_rate(2 * per_fmt, world, ms) / 1e9
     k_ms = statistics.mean(e[i][0].elapsed_time(e[i][1]) for e in evs for i in range(2))
     achieved = per_fmt / (k_ms * 1e-3) / 1e9
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -546,13 +559,10 @@ def main():
     with ClockSampler(gpu_index) as clk:
         total_ms, q_ms, g_ms, _ = time_linear_steps(torch, fp8, wl, args.steps, args.warmup, stream, barrier)
     clocks = clk.summary()
-    if dist:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
     ms_per_step = total_ms / args.steps
     flops = 2.0 * M * N * K
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, ms_per_step) / 1e12
     g_avg = statistics.mean(g_ms)
     q_avg = statistics.mean(q_ms)
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_OVER_BF16
