@@ -342,6 +342,48 @@ def extras(torch, fp8, stream, peaks):
                                "gemm_tflops": 2 * M * N * K / ((statistics.median(times_l) - qm) * 1e-3) / 1e12}
     del xs_steps, wq, y, xq
     torch.cuda.empty_cache()
+    # context: the same llama70b_prefill GEMM through cuBLASLt (torch._scaled_mm, per-row
+    # scales, bf16 out) and through fp8_scaled_gemm, each 300 launches back to back
+    try:
+        from fp8_dynamic_scaled_b200 import inputs as _inp
+        M, K, N = 4096, 8192, 28672
+        xh, wh = _inp.llama70b_prefill(M, K, N)
+        xq, xs, _ = fp8.empty_quant_outputs(M, K, fp8.FP8_SCALE_ROW)
+        wq, wsc, _ = fp8.empty_quant_outputs(N, K, fp8.FP8_SCALE_ROW)
+        fp8.fp8_quantize(to_dev_bf16(torch, xh), fp8.FP8_E4M3, fp8.FP8_SCALE_ROW, xq, xs)
+        fp8.fp8_quantize(to_dev_bf16(torch, wh), fp8.FP8_E4M3, fp8.FP8_SCALE_ROW, wq, wsc)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        a8 = xq.view(torch.float8_e4m3fn)
+        b8 = wq.view(torch.float8_e4m3fn).t()
+        sa, sb = xs.view(M, 1), wsc.view(1, N)
+
+        def run_ours():
+            fp8.fp8_scaled_gemm(xq, xs, fp8.FP8_SCALE_ROW, fp8.FP8_E4M3, wq, wsc, fp8.FP8_SCALE_ROW, fp8.FP8_E4M3, y,
+                                stream=stream)
+
+        def run_cublas():
+            torch._scaled_mm(a8, b8, scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+
+        res = {}
+        for name, fn in (("fp8_scaled_gemm", run_ours), ("cublaslt_scaled_mm", run_cublas)):
+            with torch.cuda.stream(stream):
+                for _ in range(5):
+                    fn()
+                torch.cuda.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(300):
+                    fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / 300
+            res[name] = {"us": ms * 1e3, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}
+        res["note"] = "library context only; same shapes, per-row scales, bf16 out, 300 back-to-back launches each"
+        out["gemm_vs_cublaslt"] = res
+        del xq, wq, y
+        torch.cuda.empty_cache()
+    except Exception as ex:  # the comparison is context; a missing cuBLASLt FP8 path must not fail the bench
+        out["gemm_vs_cublaslt"] = {"error": str(ex)[:200]}
     # small per-tensor linear (latency-bound)
     xh, wh = inputs.linear_small()
     x, w = to_dev_bf16(torch, xh), to_dev_bf16(torch, wh)
