@@ -71,6 +71,8 @@ def _load():
     lib.orc_f32_to_bf16_array.restype, lib.orc_f32_to_bf16_array.argtypes = None, [P, I64, P]
     lib.orc_quant_scaled_array.restype = None
     lib.orc_quant_scaled_array.argtypes = [P, I64, F, I32, P]
+    lib.orc_dequant_scaled_array.restype = None
+    lib.orc_dequant_scaled_array.argtypes = [P, I64, F, I32, P]
     _lib = lib
     return lib
 
@@ -122,6 +124,14 @@ def quant_scaled(values, s: float, fmt: int) -> np.ndarray:
     return out
 
 
+def dequant_scaled(codes, s: float, fmt: int) -> np.ndarray:
+    """bf16 bit patterns of fp32(decode(q) * s) ([FFS] "Scale 怎样把 Tensor 塞进 E4M3": X^ = s X_fp8)."""
+    q = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(q.size, np.uint16)
+    _load().orc_dequant_scaled_array(_ptr(q.ravel()), q.size, float(s), fmt, _ptr(out))
+    return out.reshape(q.shape)
+
+
 def f32_to_bf16(values) -> np.ndarray:
     v = np.ascontiguousarray(values, dtype=np.float32).ravel()
     out = np.empty(v.size, np.uint16)
@@ -171,6 +181,33 @@ def quantize(x_bf16: np.ndarray, fmt: int, mode: int, dequant: bool = True):
     if rc != 0:
         raise OracleError(f"orc_quantize failed: {rc} ({'non-finite input' if rc == 1 else 'bad argument'})")
     return q, scale, deq
+
+
+def bf16_to_f32(x_bf16: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns: the pattern is the top half of the fp32 one."""
+    return (np.asarray(x_bf16, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def amax(x_bf16: np.ndarray) -> float:
+    """a_max = max |x| over a bf16 tensor ([FFS] "Scale 怎样把 Tensor 塞进 E4M3", eq. a_max = max|X|);
+    0 for an empty tensor.  Non-finite input is rejected, as everywhere in the oracle."""
+    v = bf16_to_f32(x_bf16)
+    if v.size == 0:
+        return 0.0
+    if not np.all(np.isfinite(v)):
+        raise OracleError("non-finite input")
+    return float(np.max(np.abs(v)))
+
+
+def quantize_with_amax(x_bf16: np.ndarray, fmt: int, amax_value: float, dequant: bool = True):
+    """Per-tensor current scaling with a given a_max (the cast phase alone):
+    s = fp32(max(a_max, 1e-12f) / F_max), q = encode(clip(fp32(x / s))), X^ = bf16(fp32(decode(q) s)).
+    Returns (codes [rows, cols], s float32, dequant bf16 bits or None)."""
+    assert x_bf16.dtype == np.uint16 and x_bf16.ndim == 2
+    s = np.float32(scale_from_amax(np.float32(amax_value), fmt))
+    q = quant_scaled(bf16_to_f32(x_bf16), float(s), fmt).reshape(x_bf16.shape)
+    d = dequant_scaled(q, float(s), fmt) if dequant else None
+    return q, s, d
 
 
 def delayed_step(x_bf16: np.ndarray, fmt: int, ring: np.ndarray, t: int, dequant: bool = False):
@@ -228,6 +265,30 @@ def gemm_ref_points(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b, pm, pn):
     y[order] = ys
     bound[order] = bs
     return y, bound
+
+
+def epilogue_ref(y_ref, bound, bias_bf16=None):
+    """GEMM reference with the output bias ([PQG] code fp8_gemm_forward: bias added to the
+    scaled product before the BF16 output): y + bias[n] in fp64, and |bias[n]| added to the
+    bound of the acceptance rule."""
+    if bias_bf16 is None:
+        return y_ref, bound
+    b = bf16_to_f32(bias_bf16).astype(np.float64)
+    return y_ref + b, bound + np.abs(b)
+
+
+def requant_interval(y_ref, lim, s_y: float, fmt: int):
+    """Values an FP8 output code may decode to when the bf16 output y lies within
+    [y_ref - lim, y_ref + lim] and is then quantised with the fixed scale s_y
+    ([FFS] "一次 FP8 GEMM 的完整精度契约": output scale / requantisation for an FP8
+    consumer).  The quantiser is monotone, so the code of y lies between the codes of
+    the interval's ends.  Returns the decoded values (unscaled, i.e. before the factor
+    s_y) of the lowest and the highest admissible code, elementwise."""
+    y_ref = np.asarray(y_ref, np.float64)
+    lo = quant_scaled((y_ref - lim).astype(np.float32), s_y, fmt)
+    hi = quant_scaled((y_ref + lim).astype(np.float32), s_y, fmt)
+    table = decode_table(fmt)
+    return table[lo].reshape(y_ref.shape), table[hi].reshape(y_ref.shape)
 
 
 def bf16_ulp(y: np.ndarray) -> np.ndarray:

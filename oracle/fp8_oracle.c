@@ -495,6 +495,10 @@ void orc_f32_to_bf16_array(const float* v, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = orc_f32_to_bf16(v[i]);
 }
 /* Quantize an array of fp32 values with one fp32 scale: t = x/s, clip, encode. */
+/* Dequantised bf16 of codes under one fp32 scale: bf16_RNE(fp32(decode(q) * s)). */
+void orc_dequant_scaled_array(const uint8_t* q, int64_t n, float s, int fmt, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = dequant_one(q[i], s, fmt);
+}
 void orc_quant_scaled_array(const float* v, int64_t n, float s, int fmt, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = quant_one(v[i], s, fmt, NULL);
 }
