@@ -30,13 +30,19 @@ FP8_OK, FP8_ERR_INVALID_ARG, FP8_ERR_ALIGNMENT, FP8_ERR_UNSUPPORTED_DEVICE = 0, 
 FP8_ERR_NONFINITE, FP8_ERR_TIMEOUT, FP8_ERR_CUDA, FP8_ERR_WORKSPACE = 4, 5, 6, 7
 
 EXPORTED = ("fp8_abi_version", "fp8_status_string", "fp8_device_check", "fp8_workspace_size",
-            "fp8_quantize", "fp8_scaled_gemm", "fp8_linear_forward", "fp8_linear_forward_noalloc")
+            "fp8_quantize", "fp8_scaled_gemm", "fp8_linear_forward", "fp8_linear_forward_noalloc",
+            "fp8_amax", "fp8_quantize_with_amax", "fp8_scaled_gemm_ex", "fp8_linear_forward_ex")
 FP8_NOALLOC_SCRATCH_BYTES = 4194304
 
 
 class fp8_history_t(ctypes.Structure):
     _fields_ = [("ring_dev", ctypes.c_void_p), ("len", ctypes.c_int32), ("step", ctypes.c_int64),
                 ("pending_dev", ctypes.c_void_p), ("ticket_dev", ctypes.c_void_p)]
+
+
+class fp8_epilogue_t(ctypes.Structure):
+    _fields_ = [("bias_dev", ctypes.c_void_p), ("amax_dev", ctypes.c_void_p), ("yq_dev", ctypes.c_void_p),
+                ("yq_scale_dev", ctypes.c_void_p), ("yq_fmt", ctypes.c_int32), ("ldq", ctypes.c_int64)]
 
 
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -54,6 +60,17 @@ _lib.fp8_scaled_gemm.argtypes = [_P, _P, _I32, _I32, _P, _P, _I32, _I32, _I64, _
 _lib.fp8_linear_forward.restype = _I32
 _lib.fp8_linear_forward.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P, _P,
                                     _I32, _I32, _I64, _P, _I64, _P, _P, _SZ, _P]
+_lib.fp8_amax.restype = _I32
+_lib.fp8_amax.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]
+_lib.fp8_quantize_with_amax.restype = _I32
+_lib.fp8_quantize_with_amax.argtypes = [_P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _P]
+_lib.fp8_scaled_gemm_ex.restype = _I32
+_lib.fp8_scaled_gemm_ex.argtypes = [_P, _P, _I32, _I32, _P, _P, _I32, _I32, _I64, _I64, _I64, _P, _I64,
+                                    ctypes.POINTER(fp8_epilogue_t), _P, _P, _SZ, _P]
+_lib.fp8_linear_forward_ex.restype = _I32
+_lib.fp8_linear_forward_ex.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P, _P,
+                                       _I32, _I32, _I64, _P, _I64, ctypes.POINTER(fp8_epilogue_t), _P, _P, _SZ,
+                                       _P]
 _lib.fp8_linear_forward_noalloc.restype = _I32
 _lib.fp8_linear_forward_noalloc.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P,
                                             _P, _I32, _I32, _I64, _P, _I64, _P, _P]
@@ -164,6 +181,77 @@ def fp8_linear_forward(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, workspace
                                  w_mode, w_fmt, N, _ptr(y), ldy, _ptr(dev_status), _ptr(workspace),
                                  _nbytes(workspace), _stream(stream))
     _check(rc, "fp8_linear_forward")
+
+
+def fp8_amax(x, amax, *, dev_status=None, workspace=None, stream=None):
+    """amax[0] (device fp32) = max |x| over bf16 x [rows, cols]."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or (x.numel() and x.stride(1) != 1):
+        raise TypeError("x must be a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    rc = _lib.fp8_amax(_ptr(x), rows, cols, ld, _ptr(amax), _ptr(dev_status), _ptr(workspace), _nbytes(workspace),
+                       _stream(stream))
+    _check(rc, "fp8_amax")
+
+
+def fp8_quantize_with_amax(x, fmt, amax, q, scale, *, dequant=None, dev_status=None, stream=None):
+    """Per-tensor cast of bf16 x with the scale of a given device amax: scale[0] = max(amax, 1e-12)/F_max."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or (x.numel() and x.stride(1) != 1):
+        raise TypeError("x must be a 2-D bf16 tensor with unit column stride")
+    if q.dtype != torch.uint8:
+        raise TypeError("q must be uint8")
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    rc = _lib.fp8_quantize_with_amax(_ptr(x), rows, cols, ld, fmt, _ptr(amax), _ptr(q), _ptr(scale), _ptr(dequant),
+                                     _ptr(dev_status), _stream(stream))
+    _check(rc, "fp8_quantize_with_amax")
+
+
+def _epilogue(N, bias, amax, yq, yq_scale, yq_fmt):
+    if bias is None and amax is None and yq is None:
+        return None
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N):
+        raise TypeError("bias must be bf16 [N]")
+    ldq = 0
+    if yq is not None:
+        if yq.dtype != torch.uint8:
+            raise TypeError("yq must be uint8 codes")
+        ldq = yq.stride(0) if yq.shape[0] > 1 else yq.shape[1]
+    return fp8_epilogue_t(_ptr(bias), _ptr(amax), _ptr(yq), _ptr(yq_scale), yq_fmt, ldq)
+
+
+def fp8_scaled_gemm_ex(a, a_scale, a_mode, fmt_a, b, b_scale, b_mode, fmt_b, y, *, bias=None, amax=None, yq=None,
+                       yq_scale=None, yq_fmt=FP8_E4M3, dev_status=None, workspace=None, stream=None):
+    """fp8_scaled_gemm with the epilogue options: bias [N] (bf16), amax (device fp32, max |y| folded in),
+    yq [M, N] FP8 codes of y / yq_scale.  y may be None when yq is given."""
+    if a.dtype != torch.uint8 or b.dtype != torch.uint8 or (y is not None and y.dtype != torch.bfloat16):
+        raise TypeError("a, b must be uint8 codes and y bf16")
+    M, K = a.shape
+    N = b.shape[0]
+    ldy = 0 if y is None else (y.stride(0) if y.shape[0] > 1 else y.shape[1])
+    epi = _epilogue(N, bias, amax, yq, yq_scale, yq_fmt)
+    rc = _lib.fp8_scaled_gemm_ex(_ptr(a), _ptr(a_scale), a_mode, fmt_a, _ptr(b), _ptr(b_scale), b_mode, fmt_b,
+                                 M, N, K, _ptr(y), ldy, ctypes.byref(epi) if epi is not None else None,
+                                 _ptr(dev_status), _ptr(workspace), _nbytes(workspace), _stream(stream))
+    _check(rc, "fp8_scaled_gemm_ex")
+
+
+def fp8_linear_forward_ex(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, workspace, *, hist: History | None = None,
+                          bias=None, amax=None, yq=None, yq_scale=None, yq_fmt=FP8_E4M3, dev_status=None,
+                          stream=None):
+    """fp8_linear_forward with the epilogue options of fp8_scaled_gemm_ex."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.uint8 or (y is not None and y.dtype != torch.bfloat16):
+        raise TypeError("x bf16, w uint8 codes, y bf16")
+    M, K = x.shape
+    N = w.shape[0]
+    ldx = x.stride(0) if M > 1 else K
+    ldy = 0 if y is None else (y.stride(0) if y.shape[0] > 1 else y.shape[1])
+    epi = _epilogue(N, bias, amax, yq, yq_scale, yq_fmt)
+    rc = _lib.fp8_linear_forward_ex(_ptr(x), M, K, ldx, x_fmt, x_mode,
+                                    ctypes.byref(hist.c) if hist is not None else None, _ptr(w), _ptr(w_scale),
+                                    w_mode, w_fmt, N, _ptr(y), ldy, ctypes.byref(epi) if epi is not None else None,
+                                    _ptr(dev_status), _ptr(workspace), _nbytes(workspace), _stream(stream))
+    _check(rc, "fp8_linear_forward_ex")
 
 
 def fp8_linear_forward_noalloc(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, *, hist: History | None = None,

@@ -47,7 +47,8 @@ size_t partials_bytes() { return align_up(4 * (size_t)amax_partials_count(), 256
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA; }
 
 int32_t check_quantize_args(const void* x, int64_t rows, int64_t cols, int64_t ld, int32_t fmt, int32_t mode,
-                            const uint8_t* q, const void* scale, const fp8_history_t* hist, const void* deq) {
+                            const uint8_t* q, const void* scale, const fp8_history_t* hist, const void* deq,
+                            bool need_q = true) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (mode < FP8_SCALE_TENSOR || mode > FP8_SCALE_DELAYED) return FP8_ERR_INVALID_ARG;
     if (mode == FP8_SCALE_MX32 && fmt != FP8_E4M3) return FP8_ERR_INVALID_ARG;
@@ -57,7 +58,7 @@ int32_t check_quantize_args(const void* x, int64_t rows, int64_t cols, int64_t l
     if (mode == FP8_SCALE_MX32 && cols % 32 != 0) return FP8_ERR_INVALID_ARG;
     if (scale == nullptr && scale_bytes(mode, rows, cols) > 0) return FP8_ERR_INVALID_ARG;
     const bool empty = rows == 0 || cols == 0;
-    if (!empty && (x == nullptr || q == nullptr)) return FP8_ERR_INVALID_ARG;
+    if (!empty && (x == nullptr || (need_q && q == nullptr))) return FP8_ERR_INVALID_ARG;
     if (mode == FP8_SCALE_DELAYED) {
         if (!hist || !hist->ring_dev || !hist->pending_dev || !hist->ticket_dev || hist->len < 1 || hist->step < 0)
             return FP8_ERR_INVALID_ARG;
@@ -107,8 +108,26 @@ int32_t quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, int
     return cuda_status(launch_quantize_grouped(a, st));
 }
 
+// An epilogue descriptor with every pointer NULL is the plain GEMM.
+bool epi_active(const fp8_epilogue_t* e) {
+    return e != nullptr && (e->bias_dev != nullptr || e->amax_dev != nullptr || e->yq_dev != nullptr);
+}
+
+int32_t check_epilogue(const fp8_epilogue_t* e, int64_t N) {
+    if (!epi_active(e)) return FP8_OK;
+    if (e->yq_dev != nullptr) {
+        if (e->yq_fmt != FP8_E4M3 && e->yq_fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+        if (e->yq_scale_dev == nullptr || e->ldq < N) return FP8_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(e->yq_scale_dev) & 3u) != 0) return FP8_ERR_ALIGNMENT;
+    }
+    if (!aligned16(e->bias_dev)) return FP8_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(e->amax_dev) & 3u) != 0) return FP8_ERR_ALIGNMENT;
+    return FP8_OK;
+}
+
 int32_t check_gemm_args(const uint8_t* a, const void* sa, int32_t am, int32_t fa, const uint8_t* b, const void* sb,
-                        int32_t bm, int32_t fb, int64_t M, int64_t N, int64_t K, const void* y, int64_t ldy) {
+                        int32_t bm, int32_t fb, int64_t M, int64_t N, int64_t K, const void* y, int64_t ldy,
+                        const fp8_epilogue_t* epi = nullptr) {
     if (fa != FP8_E4M3 && fa != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (fb != FP8_E4M3 && fb != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0) return FP8_ERR_INVALID_ARG;
@@ -122,9 +141,11 @@ int32_t check_gemm_args(const uint8_t* a, const void* sa, int32_t am, int32_t fa
     const bool mx = am == FP8_SCALE_MX32 && bm == FP8_SCALE_MX32;
     if (!rowscale && !block && !mx) return FP8_ERR_INVALID_ARG;
     if (mx && (fa != FP8_E4M3 || fb != FP8_E4M3 || K % 32 != 0)) return FP8_ERR_INVALID_ARG;
-    if (ldy < N) return FP8_ERR_INVALID_ARG;
+    const bool fp8_only = y == nullptr && epi_active(epi) && epi->yq_dev != nullptr;
+    if (!fp8_only && ldy < N) return FP8_ERR_INVALID_ARG;
+    if (int32_t rc = check_epilogue(epi, N)) return rc;
     if (M > 0 && N > 0) {
-        if (y == nullptr) return FP8_ERR_INVALID_ARG;
+        if (y == nullptr && !fp8_only) return FP8_ERR_INVALID_ARG;
         if (K > 0 && (a == nullptr || b == nullptr || sa == nullptr || sb == nullptr)) return FP8_ERR_INVALID_ARG;
     }
     if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(y) & 1u) != 0) return FP8_ERR_ALIGNMENT;
@@ -134,10 +155,19 @@ int32_t check_gemm_args(const uint8_t* a, const void* sa, int32_t am, int32_t fa
 
 int32_t gemm_impl(const uint8_t* a, const void* sa, int32_t am, int32_t fa, const uint8_t* b, const void* sb,
                   int32_t bm, int32_t fb, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int32_t* status,
-                  cudaStream_t st) {
+                  cudaStream_t st, const fp8_epilogue_t* epi = nullptr) {
     if (M == 0 || N == 0) return FP8_OK;
-    if (K == 0) return cuda_status(launch_zero_output(static_cast<uint16_t*>(y), M, N, ldy, st));
+    const bool ext = epi_active(epi);
+    if (K == 0 && !ext) return cuda_status(launch_zero_output(static_cast<uint16_t*>(y), M, N, ldy, st));
     GemmArgs g{};
+    if (ext) {
+        g.bias = static_cast<const uint16_t*>(epi->bias_dev);
+        g.amax = epi->amax_dev;
+        g.yq = epi->yq_dev;
+        g.yq_scale = epi->yq_scale_dev;
+        g.yq_fmt = epi->yq_fmt;
+        g.ldq = epi->ldq;
+    }
     g.a = a;
     g.b = b;
     g.sa = sa;
@@ -152,6 +182,7 @@ int32_t gemm_impl(const uint8_t* a, const void* sa, int32_t am, int32_t fa, cons
     g.y = static_cast<uint16_t*>(y);
     g.ldy = ldy;
     g.status = status;
+    if (K == 0) return cuda_status(launch_zero_k_epilogue(g, st));
     return cuda_status(launch_gemm(g, st));
 }
 
@@ -200,6 +231,49 @@ int32_t fp8_quantize(const void* x_dev, int64_t rows, int64_t cols, int64_t ld, 
                          workspace_dev, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+int32_t fp8_amax(const void* x_dev, int64_t rows, int64_t cols, int64_t ld, float* amax_dev, int32_t* dev_status,
+                 void* workspace_dev, size_t ws_bytes, void* stream) {
+    if (amax_dev == nullptr) return FP8_ERR_INVALID_ARG;
+    int32_t rc = check_quantize_args(x_dev, rows, cols, ld, FP8_E4M3, FP8_SCALE_TENSOR, nullptr, amax_dev, nullptr,
+                                     nullptr, /*need_q=*/false);
+    if (rc != FP8_OK) return rc;
+    if ((rc = device_gate()) != FP8_OK) return rc;
+    if (workspace_dev == nullptr || ws_bytes < partials_bytes()) return FP8_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace_dev) & 3u) != 0) return FP8_ERR_ALIGNMENT;
+    QuantArgs a{};
+    a.x = static_cast<const uint16_t*>(x_dev);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.status = dev_status;
+    a.partials = static_cast<uint32_t*>(workspace_dev);
+    return cuda_status(launch_amax(a, amax_dev, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t fp8_quantize_with_amax(const void* x_dev, int64_t rows, int64_t cols, int64_t ld, int32_t fmt,
+                               const float* amax_dev, uint8_t* q_dev, float* scale_dev, void* dequant_dev,
+                               int32_t* dev_status, void* stream) {
+    if (amax_dev == nullptr || scale_dev == nullptr) return FP8_ERR_INVALID_ARG;
+    int32_t rc = check_quantize_args(x_dev, rows, cols, ld, fmt, FP8_SCALE_TENSOR, q_dev, scale_dev, nullptr,
+                                     dequant_dev);
+    if (rc != FP8_OK) return rc;
+    if ((reinterpret_cast<uintptr_t>(amax_dev) & 3u) != 0) return FP8_ERR_ALIGNMENT;
+    if ((rc = device_gate()) != FP8_OK) return rc;
+    QuantArgs a{};
+    a.x = static_cast<const uint16_t*>(x_dev);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.fmt = fmt;
+    a.mode = FP8_SCALE_TENSOR;
+    a.q = q_dev;
+    a.scale = scale_dev;
+    a.deq = static_cast<uint16_t*>(dequant_dev);
+    a.status = dev_status;
+    a.amax_in = amax_dev;
+    return cuda_status(launch_quantize_given(a, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t fp8_scaled_gemm(const uint8_t* a_dev, const void* a_scale_dev, int32_t a_mode, int32_t fmt_a,
                         const uint8_t* b_dev, const void* b_scale_dev, int32_t b_mode, int32_t fmt_b, int64_t M,
                         int64_t N, int64_t K, void* y_dev, int64_t ldy, int32_t* dev_status, void* workspace_dev,
@@ -214,10 +288,24 @@ int32_t fp8_scaled_gemm(const uint8_t* a_dev, const void* a_scale_dev, int32_t a
                      dev_status, static_cast<cudaStream_t>(stream));
 }
 
-int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt, int32_t x_mode,
+int32_t fp8_scaled_gemm_ex(const uint8_t* a_dev, const void* a_scale_dev, int32_t a_mode, int32_t fmt_a,
+                           const uint8_t* b_dev, const void* b_scale_dev, int32_t b_mode, int32_t fmt_b, int64_t M,
+                           int64_t N, int64_t K, void* y_dev, int64_t ldy, const fp8_epilogue_t* epi,
+                           int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream) {
+    (void)workspace_dev;
+    (void)ws_bytes;
+    int32_t rc = check_gemm_args(a_dev, a_scale_dev, a_mode, fmt_a, b_dev, b_scale_dev, b_mode, fmt_b, M, N, K, y_dev,
+                                 ldy, epi);
+    if (rc != FP8_OK) return rc;
+    if ((rc = device_gate()) != FP8_OK) return rc;
+    return gemm_impl(a_dev, a_scale_dev, a_mode, fmt_a, b_dev, b_scale_dev, b_mode, fmt_b, M, N, K, y_dev, ldy,
+                     dev_status, static_cast<cudaStream_t>(stream), epi);
+}
+
+int32_t fp8_linear_forward_ex(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt, int32_t x_mode,
                            fp8_history_t* hist, const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
-                           int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy, int32_t* dev_status,
-                           void* workspace_dev, size_t ws_bytes, void* stream) {
+                              int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy, const fp8_epilogue_t* epi,
+                              int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream) {
     if (x_mode == FP8_SCALE_BLOCK_128x128) return FP8_ERR_INVALID_ARG;   // activations use 1x128 blocks
     const size_t need = fp8_workspace_size(2, M, N, K, x_mode);
     if (need == 0) return FP8_ERR_INVALID_ARG;
@@ -230,13 +318,21 @@ int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int64_t ldx,
     int32_t rc = check_quantize_args(x_dev, M, K, ldx, x_fmt, x_mode, xq, xs, hist, nullptr);
     if (rc != FP8_OK) return rc;
     const int32_t gm_a = x_mode == FP8_SCALE_DELAYED ? FP8_SCALE_TENSOR : x_mode;
-    rc = check_gemm_args(xq, xs, gm_a, x_fmt, w_dev, w_scale_dev, w_mode, w_fmt, M, N, K, y_dev, ldy);
+    rc = check_gemm_args(xq, xs, gm_a, x_fmt, w_dev, w_scale_dev, w_mode, w_fmt, M, N, K, y_dev, ldy, epi);
     if (rc != FP8_OK) return rc;
     if ((rc = device_gate()) != FP8_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = quantize_impl(x_dev, M, K, ldx, x_fmt, x_mode, xq, xs, hist, nullptr, dev_status, part, partials_bytes(), st);
     if (rc != FP8_OK) return rc;
-    return gemm_impl(xq, xs, gm_a, x_fmt, w_dev, w_scale_dev, w_mode, w_fmt, M, N, K, y_dev, ldy, dev_status, st);
+    return gemm_impl(xq, xs, gm_a, x_fmt, w_dev, w_scale_dev, w_mode, w_fmt, M, N, K, y_dev, ldy, dev_status, st, epi);
+}
+
+int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt, int32_t x_mode,
+                           fp8_history_t* hist, const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
+                           int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy, int32_t* dev_status,
+                           void* workspace_dev, size_t ws_bytes, void* stream) {
+    return fp8_linear_forward_ex(x_dev, M, K, ldx, x_fmt, x_mode, hist, w_dev, w_scale_dev, w_mode, w_fmt, N, y_dev,
+                                 ldy, nullptr, dev_status, workspace_dev, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -72,6 +72,22 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
     return d;
 }
 
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(reinterpret_cast<unsigned long long&>(d))
+        : "l"(reinterpret_cast<const unsigned long long&>(a)), "l"(reinterpret_cast<const unsigned long long&>(b)));
+    return d;
+}
+
+// Lane-wise clamp of a packed bf16 pair to [lo, hi] (both packed pairs).
+__device__ __forceinline__ uint32_t clamp_bf16x2(uint32_t v, uint32_t lo, uint32_t hi) {
+    uint32_t d;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(hi));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(d), "r"(lo));
+    return d;
+}
+
 // ---------------------------------------------------------------- FP8 casts
 // Two fp32 values -> two codes (a in the low byte), round-to-nearest-even with
 // saturation to the largest finite value: for finite inputs identical to

@@ -102,6 +102,16 @@ struct GemmParams {
     uint16_t* y;
     int64_t ldy;
     int32_t y_direct;
+    // optional epilogue (fp8_epilogue_t); ext != 0 when any option is set
+    int32_t ext;
+    int32_t write_y;        // 0: no bf16 Y (FP8 output only)
+    const uint16_t* bias;   // bf16 [N], 16-byte aligned, or null
+    uint32_t* amax;         // fp32 bit pattern folded with atomicMax, or null
+    uint8_t* yq;            // FP8 codes [M, ldq], or null
+    const float* yq_scale;
+    int64_t ldq;
+    int32_t yq_fmt;
+    int32_t yq_vec;         // yq rows start 16-byte aligned
 };
 
 // ---------------------------------------------------------------- bounded waits
@@ -173,8 +183,138 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap* tmY, uint8_t* buf
     }
 }
 
+// ---------------------------------------------------------------- optional epilogue
+// Per-lane state of the fp8_epilogue_t options: the running |y| maximum and the
+// constants of the FP8 output cast y_q = RNE(clip(y / s_y)).
+struct EpiState {
+    uint32_t amax2;        // packed |bf16| maxima (sign bits meaningless)
+    float2 s2, nr2;        // s_y and -1/s_y in both lanes
+    uint32_t lo2, hi2;     // clip bounds of y as packed bf16 pairs
+    bool yq_ok;
+};
+
+__device__ __forceinline__ EpiState epi_init(const GemmParams& p) {
+    EpiState e;
+    e.amax2 = 0;
+    e.s2 = e.nr2 = make_float2(0.0f, 0.0f);
+    e.lo2 = e.hi2 = 0;
+    e.yq_ok = false;
+    if (p.ext && p.yq) {
+        const float s = __ldg(p.yq_scale);
+        // s and 1/s both normal: 2^-126 <= s <= 2^126
+        e.yq_ok = s >= 1.17549435e-38f && s <= 8.5070592e37f;
+        if (!e.yq_ok && (threadIdx.x & 31) == 0) report_status(p.status, FP8_ERR_INVALID_ARG);
+        if (e.yq_ok) {
+            const float r = __frcp_rn(s);
+            e.s2 = make_float2(s, s);
+            e.nr2 = make_float2(-r, -r);
+            // y / s_y is computed as a reciprocal with one Markstein correction, exact
+            // (as IEEE division) while y * (1/s_y) stays finite.  |y| is first clipped
+            // to the largest bf16 <= 2^127 s_y: anything beyond saturates either way.
+            const uint32_t lim = min(__float_as_uint(__fmul_rn(s, 1.7014118e38f)) >> 16, 0x7F7Fu);
+            e.hi2 = lim | (lim << 16);
+            e.lo2 = e.hi2 | 0x80008000u;
+        }
+    }
+    return e;
+}
+
+// The options on 32 columns [n0, n0 + 32) of one output row held by this lane:
+// f[] are the scaled fp32 accumulators.  Adds the bias, rounds to bf16 (w, for the
+// Y store), folds |y| into the running maximum and writes the FP8 output codes.
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, EpiState& es, float (&f)[32], int32_t n0,
+                                          int32_t row, uint32_t (&w)[16]) {
+    if (p.bias) {
+        if (n0 + 32 <= p.N) {
+            const uint4* b4 = reinterpret_cast<const uint4*>(p.bias + n0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 b = __ldg(b4 + q);
+                const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 s = add2_rn(make_float2(f[8 * q + 2 * i], f[8 * q + 2 * i + 1]),
+                                             make_float2(bf16_lo(bw[i]), bf16_hi(bw[i])));
+                    f[8 * q + 2 * i] = s.x;
+                    f[8 * q + 2 * i + 1] = s.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float b = n0 + j < p.N ? bf16bits_to_float(__ldg(p.bias + n0 + j)) : 0.0f;
+                f[j] = __fadd_rn(f[j], b);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+    if (row >= p.M) return;
+    if (p.amax) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) es.amax2 = bmax_abs_bf16x2(es.amax2, w[j]);
+    }
+    if (es.yq_ok) {
+        uint32_t c[8];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            // on -y with -1/s_y: q = RN(y r), e = -(y - q s) exactly, t = RN(q + (y - q s) r);
+            // keeps the sign of a zero y
+            const uint32_t wn = clamp_bf16x2(w[j], es.lo2, es.hi2) ^ 0x80008000u;
+            const float2 nx = make_float2(__uint_as_float(wn << 16), __uint_as_float(wn & 0xFFFF0000u));
+            const float2 q = mul2_rn(nx, es.nr2);
+            const float2 e = fma2_rn(q, es.s2, nx);
+            const float2 t = fma2_rn(e, es.nr2, q);
+            const uint32_t code = p.yq_fmt == FP8_E4M3 ? cvt_pair<FP8_E4M3>(t.x, t.y) : cvt_pair<FP8_E5M2>(t.x, t.y);
+            c[j / 2] = (j & 1) ? (c[j / 2] | (code << 16)) : code;
+        }
+        uint8_t* dst = p.yq + (int64_t)row * p.ldq + n0;
+        if (n0 + 32 <= p.N && p.yq_vec) {
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(c[0], c[1], c[2], c[3]);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (n0 + j < p.N) dst[j] = (uint8_t)(c[j / 4] >> (8 * (j & 3)));
+        }
+    }
+}
+
+// End of a warp's epilogue: fold its |y| maximum into the caller's amax.
+__device__ __forceinline__ void epi_flush(const GemmParams& p, const EpiState& es, int lane) {
+    if (!p.amax) return;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, hmax_pair(es.amax2 & 0x7FFF7FFFu));
+    // |y| >= 0: the fp32 bit pattern (bf16 pattern << 16) orders like the value
+    if (lane == 0 && m != 0) atomicMax(p.amax, m << 16);
+}
+
+// Per-tensor / per-row scales on 32 accumulator columns of one row:
+// y = acc * (s_a[m] * s_b[n]), then the plain bf16 rounding or the options.
+template <bool EXT>
+__device__ __forceinline__ void rowscale_chunk(const GemmParams& p, EpiState& es, const uint32_t (&r)[32], float sx,
+                                               int32_t n0, int32_t row, uint32_t (&w)[16]) {
+    if constexpr (!EXT) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+            const int32_t n = n0 + j;
+            const float s0 = n < p.N ? sx * __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
+            const float s1 = n + 1 < p.N ? sx * __ldg(p.sb + (int64_t)(n + 1) * p.sb_stride) : 0.0f;
+            w[j / 2] = pack_bf16x2(__uint_as_float(r[j]) * s0, __uint_as_float(r[j + 1]) * s1);
+        }
+    } else {
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int32_t n = n0 + j;
+            const float s = n < p.N ? sx * __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
+            f[j] = __uint_as_float(r[j]) * s;
+        }
+        epi_chunk(p, es, f, n0, row, w);
+    }
+}
+
 // ================================================================ the kernel
-template <int V>
+template <int V, bool EXT>
 __global__ void __launch_bounds__(Smem<V>::NT, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -409,6 +549,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         uint32_t acc_it = 0;
         uint32_t store_it = 0;
         bool ok = true;
+        EpiState es;
+        if (EXT) es = epi_init(p);
         for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             int32_t mb, nb;
             tile_coords(p, t, mb, nb);
@@ -431,14 +573,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
                     const int32_t n0 = nb * BN + c * 32;
                     uint32_t w[16];
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const int32_t n = n0 + j;
-                        const float s0 = n < p.N ? sx * __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
-                        const float s1 = n + 1 < p.N ? sx * __ldg(p.sb + (int64_t)(n + 1) * p.sb_stride) : 0.0f;
-                        w[j / 2] = pack_bf16x2(__uint_as_float(r[j]) * s0, __uint_as_float(r[j + 1]) * s1);
-                    }
-                    if (n0 < p.N) {
+                    rowscale_chunk<EXT>(p, es, r, sx, n0, row, w);
+                    if (n0 < p.N && (!EXT || p.write_y)) {
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
                         __syncwarp();
@@ -514,9 +650,19 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 for (int c = 0; c < 4; ++c) {
                     const int32_t n0 = nb * BN + half * 128 + c * 32;
                     uint32_t w[16];
+                    if (!EXT) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(acc[c * 16 + j].x, acc[c * 16 + j].y);
-                    if (n0 < p.N) {
+                        for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(acc[c * 16 + j].x, acc[c * 16 + j].y);
+                    } else {
+                        float f[32];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            f[2 * j] = acc[c * 16 + j].x;
+                            f[2 * j + 1] = acc[c * 16 + j].y;
+                        }
+                        epi_chunk(p, es, f, n0, row, w);
+                    }
+                    if (n0 < p.N && (!EXT || p.write_y)) {
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
                         __syncwarp();
@@ -540,10 +686,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 for (int c = 0; c < 4; ++c) {
                     const int32_t n0 = nb * BN + half * 128 + c * 32;
                     uint32_t w[16];
+                    if (!EXT) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2)
-                        w[j / 2] = pack_bf16x2(__uint_as_float(r[c][j]), __uint_as_float(r[c][j + 1]));
-                    if (n0 < p.N) {
+                        for (int j = 0; j < 32; j += 2)
+                            w[j / 2] = pack_bf16x2(__uint_as_float(r[c][j]), __uint_as_float(r[c][j + 1]));
+                    } else {
+                        float f[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[c][j]);
+                        epi_chunk(p, es, f, n0, row, w);
+                    }
+                    if (n0 < p.N && (!EXT || p.write_y)) {
                         uint8_t* b = ybuf + (store_it % C::STAGE_BUFS) * 2048;
                         if (lane == 0) ptx::bulk_wait_read<C::STAGE_BUFS - 1>();
                         __syncwarp();
@@ -553,6 +706,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
             }
         }
+        if (EXT) epi_flush(p, es, lane);     // every lane reaches this point
         if (lane == 0) ptx::bulk_wait_all();
         __syncwarp();
     }
@@ -594,6 +748,7 @@ struct PairSmem {
     static constexpr uint32_t ALLOC = TOTAL + 1024;
 };
 
+template <bool EXT>
 __global__ void __launch_bounds__(PairSmem::NT, 1)
 fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -720,6 +875,8 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         uint8_t* ybuf = sY + ew * S::STAGE_BUFS * 2048;
         uint32_t acc_it = 0, store_it = 0;
         bool ok = true;
+        EpiState es;
+        if (EXT) es = epi_init(p);
         for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
             int32_t mb, nb;
             tile_coords(p, t, mb, nb);
@@ -741,14 +898,8 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 }
                 const int32_t n0 = nb * BN + c * 32;
                 uint32_t w[16];
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const int32_t n = n0 + j;
-                    const float s0 = n < p.N ? sx * __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
-                    const float s1 = n + 1 < p.N ? sx * __ldg(p.sb + (int64_t)(n + 1) * p.sb_stride) : 0.0f;
-                    w[j / 2] = pack_bf16x2(__uint_as_float(r[j]) * s0, __uint_as_float(r[j + 1]) * s1);
-                }
-                if (n0 < p.N) {
+                rowscale_chunk<EXT>(p, es, r, sx, n0, row, w);
+                if (n0 < p.N && (!EXT || p.write_y)) {
                     uint8_t* b = ybuf + (store_it % S::STAGE_BUFS) * 2048;
                     if (lane == 0) ptx::bulk_wait_read<S::STAGE_BUFS - 1>();
                     __syncwarp();
@@ -758,6 +909,7 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             }
             ++acc_it;
         }
+        if (EXT) epi_flush(p, es, lane);     // every lane reaches this point
         if (lane == 0) ptx::bulk_wait_all();
         __syncwarp();
     }
@@ -811,7 +963,7 @@ static int num_sms() {
     return n;
 }
 
-template <int V>
+template <int V, bool EXT>
 static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaStream_t st) {
     CUtensorMap ta, tb, ty;
     // M, N, K sizes beyond 2^31 are rejected by the API before this point.
@@ -826,14 +978,14 @@ static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaSt
         return cudaErrorInvalidValue;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<V, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)Smem<V>::ALLOC);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
     const int32_t tiles = p.num_m * p.num_n;
     const int grid = std::max(1, std::min(tiles, num_sms()));
-    fp8_gemm_kernel<V><<<grid, Smem<V>::NT, Smem<V>::ALLOC, st>>>(ta, tb, ty, p);
+    fp8_gemm_kernel<V, EXT><<<grid, Smem<V>::NT, Smem<V>::ALLOC, st>>>(ta, tb, ty, p);
     return cudaGetLastError();
 }
 
@@ -846,6 +998,7 @@ static int32_t raster_group(int64_t nfast, int64_t panel_bytes) {
 }
 
 // CTA-pair launch: clusters of two CTAs, 256 x 256 tiles.
+template <bool EXT>
 static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st) {
     p.num_m = (int32_t)((g.M + P_BM - 1) / P_BM);
     p.m_fastest = (g.M <= g.N) ? 1 : 0;
@@ -863,7 +1016,7 @@ static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st)
         return cudaErrorInvalidValue;
     static int max_clusters = 0;
     if (max_clusters == 0) {
-        cudaError_t e = cudaFuncSetAttribute(fp8_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(fp8_gemm_pair_kernel<EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)PairSmem::ALLOC);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t q = {};
@@ -878,7 +1031,7 @@ static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st)
         q.attrs = qa;
         q.numAttrs = 1;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_pair_kernel, &q);
+        e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_pair_kernel<EXT>, &q);
         if (e != cudaSuccess || n <= 0) n = num_sms() / 2;
         max_clusters = n;
     }
@@ -896,7 +1049,7 @@ static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_pair_kernel, ta, tb, ty, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_pair_kernel<EXT>, ta, tb, ty, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -912,6 +1065,21 @@ static uint32_t idesc_f8f6f4(int fa, int fb) {
 static uint32_t idesc_mx(int fa, int fb) {
     return ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
            ((uint32_t)(BM >> 4) << 24);
+}
+
+// Copy the epilogue options into the kernel parameters.  Without a bf16 Y the
+// store path is never taken and no tensor map is made for it.
+static void set_epilogue(const GemmArgs& g, GemmParams& p) {
+    p.bias = g.bias;
+    p.amax = reinterpret_cast<uint32_t*>(g.amax);
+    p.yq = g.yq;
+    p.yq_scale = g.yq_scale;
+    p.yq_fmt = g.yq_fmt;
+    p.ldq = g.ldq;
+    p.yq_vec = (g.yq != nullptr && (reinterpret_cast<uintptr_t>(g.yq) & 15u) == 0 && g.ldq % 16 == 0) ? 1 : 0;
+    p.ext = (g.bias != nullptr || g.amax != nullptr || g.yq != nullptr) ? 1 : 0;
+    p.write_y = g.y != nullptr ? 1 : 0;
+    if (!p.write_y) p.y_direct = 1;
 }
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
@@ -930,6 +1098,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
     p.y = g.y;
     p.ldy = g.ldy;
     p.y_direct = (g.ldy % 8 != 0 || (reinterpret_cast<uintptr_t>(g.y) & 15u) != 0) ? 1 : 0;
+    set_epilogue(g, p);
     const bool a_pt = g.a_mode == FP8_SCALE_TENSOR || g.a_mode == FP8_SCALE_DELAYED;
     const bool b_pt = g.b_mode == FP8_SCALE_TENSOR || g.b_mode == FP8_SCALE_DELAYED;
     if ((a_pt || g.a_mode == FP8_SCALE_ROW) && (b_pt || g.b_mode == FP8_SCALE_ROW)) {
@@ -939,20 +1108,20 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
         p.sb_stride = b_pt ? 0 : 1;
         p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
         // CTA pairs once M spans a 256-row tile; a single CTA per tile below that
-        if (g.M >= P_BM) return launch_pair(g, p, st);
-        return launch_variant<V_ROWSCALE>(g, p, st);
+        if (g.M >= P_BM) return p.ext ? launch_pair<true>(g, p, st) : launch_pair<false>(g, p, st);
+        return p.ext ? launch_variant<V_ROWSCALE, true>(g, p, st) : launch_variant<V_ROWSCALE, false>(g, p, st);
     }
     if (g.a_mode == FP8_SCALE_BLOCK_1x128 && g.b_mode == FP8_SCALE_BLOCK_128x128) {
         p.sa = static_cast<const float*>(g.sa);
         p.sb = static_cast<const float*>(g.sb);
         p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
-        return launch_variant<V_BLOCK>(g, p, st);
+        return p.ext ? launch_variant<V_BLOCK, true>(g, p, st) : launch_variant<V_BLOCK, false>(g, p, st);
     }
     if (g.a_mode == FP8_SCALE_MX32 && g.b_mode == FP8_SCALE_MX32) {
         p.sfa = static_cast<const uint8_t*>(g.sa);
         p.sfb = static_cast<const uint8_t*>(g.sb);
         p.idesc = idesc_mx(g.fmt_a, g.fmt_b);
-        return launch_variant<V_MX>(g, p, st);
+        return p.ext ? launch_variant<V_MX, true>(g, p, st) : launch_variant<V_MX, false>(g, p, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -961,6 +1130,51 @@ __global__ void zero_rows_kernel(uint16_t* y, int64_t M, int64_t N, int64_t ldy)
     for (int64_t r = blockIdx.y; r < M; r += gridDim.y)
         for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < N; c += (int64_t)gridDim.x * blockDim.x)
             y[r * ldy + c] = 0;
+}
+
+// K == 0 with epilogue options: every accumulator is 0, so y = bf16(0 + bias[n]).
+// One thread per (row, 32-column chunk), the same per-lane epilogue as the GEMM.
+__global__ void __launch_bounds__(256) epi_zero_k_kernel(const GemmParams p) {
+    EpiState es = epi_init(p);
+    const int lane = threadIdx.x & 31;
+    const int64_t chunks = ((int64_t)p.N + 31) / 32;
+    const int64_t total = (int64_t)p.M * chunks;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < total; base += stride) {
+        const int64_t t = base + threadIdx.x;
+        const int32_t row = (int32_t)(t < total ? t / chunks : p.M);
+        const int32_t n0 = (int32_t)(t < total ? (t % chunks) * 32 : 0);
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = 0.0f;
+        uint32_t w[16];
+        epi_chunk(p, es, f, n0, row, w);
+        if (p.write_y && row < p.M) {
+            uint16_t* dst = p.y + (int64_t)row * p.ldy;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int32_t n = n0 + 2 * j;
+                if (n < p.N) dst[n] = (uint16_t)(w[j] & 0xFFFFu);
+                if (n + 1 < p.N) dst[n + 1] = (uint16_t)(w[j] >> 16);
+            }
+        }
+    }
+    epi_flush(p, es, lane);
+}
+
+cudaError_t launch_zero_k_epilogue(const GemmArgs& g, cudaStream_t st) {
+    GemmParams p{};
+    p.M = (int32_t)g.M;
+    p.N = (int32_t)g.N;
+    p.K = 0;
+    p.status = g.status;
+    p.y = g.y;
+    p.ldy = g.ldy;
+    set_epilogue(g, p);
+    const int64_t total = g.M * ((g.N + 31) / 32);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 8));
+    epi_zero_k_kernel<<<grid, 256, 0, st>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_zero_output(uint16_t* y, int64_t M, int64_t N, int64_t ldy, cudaStream_t st) {

@@ -24,12 +24,16 @@ struct QuantArgs {
     int64_t hist_step;
     float* hist_pending;
     uint32_t* hist_ticket;
+    // per-tensor cast with a caller's amax (launch_quantize_given)
+    const float* amax_in;
 };
 
 int32_t amax_partials_count();
 cudaError_t launch_quantize_tensor(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_quantize_grouped(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_fill_scale(float* s, int64_t n, float v, cudaStream_t st);
+cudaError_t launch_amax(const QuantArgs& a, float* out, cudaStream_t st);
+cudaError_t launch_quantize_given(const QuantArgs& a, cudaStream_t st);
 
 struct GemmArgs {
     const uint8_t* a;        // [M, K] codes
@@ -39,12 +43,20 @@ struct GemmArgs {
     int32_t a_mode, b_mode;  // TENSOR/ROW (any mix), BLOCK pair, or MX32 pair
     int32_t fmt_a, fmt_b;
     int64_t M, N, K;
-    uint16_t* y;             // bf16 [M, N], row stride ldy
+    uint16_t* y;             // bf16 [M, N], row stride ldy (null: FP8 output only)
     int64_t ldy;
     int32_t* status;
+    // epilogue options (all null: plain bf16 output)
+    const uint16_t* bias;    // bf16 [N]
+    float* amax;             // running max |y|
+    uint8_t* yq;             // FP8 codes [M, ldq]
+    const float* yq_scale;   // s_y
+    int32_t yq_fmt;
+    int64_t ldq;
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
 cudaError_t launch_zero_output(uint16_t* y, int64_t M, int64_t N, int64_t ldy, cudaStream_t st);
+cudaError_t launch_zero_k_epilogue(const GemmArgs& g, cudaStream_t st);
 
 }  // namespace fp8b

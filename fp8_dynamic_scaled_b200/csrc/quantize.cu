@@ -104,6 +104,17 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red /* [
     return r;
 }
 
+// A caller-supplied amax (fp8_quantize_with_amax): NaN or +Inf is reported and
+// replaced by the largest finite fp32 so that the scale stays finite.
+__device__ __forceinline__ float given_amax(const float* a, int32_t* status) {
+    float v = *a;
+    if (!(v <= 3.402823466e38f)) {
+        if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) report_status(status, FP8_ERR_NONFINITE);
+        v = 3.402823466e38f;
+    }
+    return v;
+}
+
 // ================================================================ per-tensor
 // Phase 1: each CTA writes the max |bf16| pattern over its share of the tensor.
 // The tensor is viewed as nrows rows of nvec 16-byte vectors (a dense tensor is
@@ -138,7 +149,8 @@ __global__ void __launch_bounds__(QT) amax_partials_kernel(const uint16_t* __res
 //   SRC_RING:     s from max(ring); the CTAs also reduce amax_t of this input
 //                 into *pending and the last CTA to finish (ticket) commits it to
 //                 ring[slot] and rearms pending/ticket.
-enum { SRC_PARTIALS = 0, SRC_RING = 1 };
+//   SRC_GIVEN:    s from a caller's amax (ring[0]); the cast checks for non-finite input.
+enum { SRC_PARTIALS = 0, SRC_RING = 1, SRC_GIVEN = 2 };
 
 template <int FMT, bool DEQ, int SRC>
 __global__ void __launch_bounds__(QT) cast_tensor_kernel(
@@ -152,10 +164,10 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
     uint32_t src = 0;
     if (SRC == SRC_PARTIALS) {
         for (int i = threadIdx.x; i < npartials; i += QT) src = max(src, partials[i]);
-    } else {
+    } else if (SRC == SRC_RING) {
         for (int i = threadIdx.x; i < ring_len; i += QT) src = max(src, __float_as_uint(ring[i]));
     }
-    src = block_max_u32(src, red);
+    if (SRC != SRC_GIVEN) src = block_max_u32(src, red);
     float amax;
     if (SRC == SRC_PARTIALS) {
         if (src >= 0x7F80u) {
@@ -163,14 +175,17 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
             src = 0x7F7Fu;     // keep the scale finite; outputs are unspecified then
         }
         amax = bf16bits_to_float(src);
-    } else {
+    } else if (SRC == SRC_RING) {
         amax = __uint_as_float(src);
+    } else {
+        amax = given_amax(ring, status);
     }
     const DivScale op{scale_from_amax<FMT>(amax)};
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         scale_out[0] = op.s;
         if (SRC == SRC_PARTIALS && ring != nullptr) ring[slot] = amax;
     }
+    constexpr bool CHECK = SRC != SRC_PARTIALS;   // inputs not already scanned by phase 1
     // ---- the cast
     uint32_t m2 = 0;
     const int64_t stride = (int64_t)gridDim.x * QT;
@@ -182,7 +197,7 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
         for (; v + stride < nvec; v += 2 * stride) {
             uint4 a = ld_v4(row + v * VEC);
             uint4 b = ld_v4(row + (v + stride) * VEC);
-            if (SRC == SRC_RING) m2 = max_bf16x2_bits(m2, max_bf16x2_bits(vec_amax2(a), vec_amax2(b)));
+            if (CHECK) m2 = max_bf16x2_bits(m2, max_bf16x2_bits(vec_amax2(a), vec_amax2(b)));
             uint2 ca = cast_vec<FMT>(a, op), cb = cast_vec<FMT>(b, op);
             *reinterpret_cast<uint2*>(qrow + v * VEC) = ca;
             *reinterpret_cast<uint2*>(qrow + (v + stride) * VEC) = cb;
@@ -193,11 +208,15 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
         }
         for (; v < nvec; v += stride) {
             uint4 a = ld_v4(row + v * VEC);
-            if (SRC == SRC_RING) m2 = max_bf16x2_bits(m2, vec_amax2(a));
+            if (CHECK) m2 = max_bf16x2_bits(m2, vec_amax2(a));
             uint2 ca = cast_vec<FMT>(a, op);
             *reinterpret_cast<uint2*>(qrow + v * VEC) = ca;
             if (DEQ) st_v4_stream(drow + v * VEC, dequant_vec<FMT>(ca, op.s));
         }
+    }
+    if (SRC == SRC_GIVEN) {
+        const uint32_t m = block_max_u32(hmax_pair(m2), red);
+        if (threadIdx.x == 0 && m >= 0x7F80u) report_status(status, FP8_ERR_NONFINITE);
     }
     if (SRC == SRC_RING) {
         uint32_t m = block_max_u32(hmax_pair(m2), red);
@@ -410,7 +429,8 @@ __global__ void __launch_bounds__(QT) quant_block128_kernel(const uint16_t* __re
 // processor", IBM J. Res. Dev. 34(1), 1990).  Quotients below the normal range
 // (|t| < 2^-126) may differ in their last bits, but every such t encodes to a
 // signed zero in both FP8 formats.
-enum { RQ_ROW = 0, RQ_B128 = 1, RQ_MX = 2, RQ_AMAX = 3, RQ_CAST = 4, RQ_DELAYED = 5 };
+//   RQ_GIVEN    per-tensor cast with a caller's amax (fp8_quantize_with_amax)
+enum { RQ_ROW = 0, RQ_B128 = 1, RQ_MX = 2, RQ_AMAX = 3, RQ_CAST = 4, RQ_DELAYED = 5, RQ_GIVEN = 6 };
 
 struct RcpScale {
     float s, r;
@@ -514,6 +534,7 @@ struct RQParams {
     int32_t slot;
     float* pending;
     uint32_t* ticket;
+    const float* amax_in;   // RQ_GIVEN
 };
 
 // One CTA per row; the row (<= QT * VPT vectors) is held in registers.
@@ -614,16 +635,18 @@ __global__ void __launch_bounds__(QT, 8) rq_amax_kernel(const RQParams p) {
 }
 
 // Per-tensor phase 2 (RQ_CAST) or the delayed single pass (RQ_DELAYED).
+// (The delayed and given-amax kinds also carry the overflow-safe cast: 5 CTAs/SM
+// leave them 48 registers.)
 template <int FMT, bool DEQ, int KIND, int U>
-__global__ void __launch_bounds__(QT, 6) rq_tensor_kernel(const RQParams p) {
+__global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(const RQParams p) {
     __shared__ uint32_t red[32];
     uint32_t src = 0;
     if (KIND == RQ_CAST) {
         for (int i = threadIdx.x; i < p.npartials; i += QT) src = max(src, p.partials[i]);
-    } else {
+    } else if (KIND == RQ_DELAYED) {
         for (int i = threadIdx.x; i < p.ring_len; i += QT) src = max(src, __float_as_uint(p.ring[i]));
     }
-    src = block_max_u32(src, red);
+    if (KIND != RQ_GIVEN) src = block_max_u32(src, red);
     float amax;
     if (KIND == RQ_CAST) {
         if (src >= 0x7F80u) {
@@ -631,11 +654,18 @@ __global__ void __launch_bounds__(QT, 6) rq_tensor_kernel(const RQParams p) {
             src = 0x7F7Fu;
         }
         amax = bf16bits_to_float(src);
-    } else {
+    } else if (KIND == RQ_DELAYED) {
         amax = __uint_as_float(src);
+    } else {
+        amax = given_amax(p.amax_in, p.status);
     }
     const float s = scale_from_amax<FMT>(amax);
     const RcpScale op{s, __frcp_rn(s)};
+    // With a scale not derived from this input (history, caller), x * (1/s) can
+    // overflow fp32; the corrected reciprocal path is exact as long as it does not.
+    // Vectors whose |x| stays below 2^127 * s (as a bf16 pattern, rounded down)
+    // take it; the rest take the overflow-safe path.
+    const uint32_t fast_lim = min(__float_as_uint(__fmul_rn(s, 1.7014118e38f)) >> 16, 0x7F7Fu);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         reinterpret_cast<float*>(p.scale)[0] = s;
         if (KIND == RQ_CAST && p.ring != nullptr) p.ring[p.slot] = amax;
@@ -646,9 +676,10 @@ __global__ void __launch_bounds__(QT, 6) rq_tensor_kernel(const RQParams p) {
     auto vec_of = [&](int64_t t) -> int64_t { return KIND == RQ_CAST ? nvec - 1 - t : t; };
     auto emit = [&](int64_t vv, const uint4& a) {
         uint2 cq;
-        if (KIND == RQ_DELAYED) {
-            m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(a));
-            cq = cast_vec_rcp_guarded<FMT>(a, op);
+        if (KIND == RQ_DELAYED || KIND == RQ_GIVEN) {
+            const uint32_t va = vec_amax2_bf(a);
+            m2 = bmax_abs_bf16x2(m2, va);
+            cq = hmax_pair(va & 0x7FFF7FFFu) <= fast_lim ? cast_vec_rcp<FMT>(a, op) : cast_vec_rcp_guarded<FMT>(a, op);
         } else {
             cq = cast_vec_rcp<FMT>(a, op);
         }
@@ -664,6 +695,10 @@ __global__ void __launch_bounds__(QT, 6) rq_tensor_kernel(const RQParams p) {
         for (int u = 0; u < U; ++u) emit(vec_of(t + u * stride), a[u]);
     }
     for (; t < nvec; t += stride) emit(vec_of(t), ld_v4(p.x + vec_of(t) * VEC));
+    if (KIND == RQ_GIVEN) {
+        const uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
+        if (threadIdx.x == 0 && m >= 0x7F80u) report_status(p.status, FP8_ERR_NONFINITE);
+    }
     if (KIND == RQ_DELAYED) {
         const uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
         if (threadIdx.x == 0) {
@@ -714,6 +749,10 @@ static void launch_cast_tensor(const QuantArgs& a, int src, dim3 grid, int npart
     if (src == SRC_PARTIALS)
         cast_tensor_kernel<FMT, DEQ, SRC_PARTIALS><<<grid, QT, 0, st>>>(
             a.x, nrows, nvec, ld, a.partials, npart, ring, len, slot, pending, ticket, a.q,
+            (float*)a.scale, a.deq, a.status);
+    else if (src == SRC_GIVEN)
+        cast_tensor_kernel<FMT, DEQ, SRC_GIVEN><<<grid, QT, 0, st>>>(
+            a.x, nrows, nvec, ld, nullptr, 0, const_cast<float*>(a.amax_in), 1, 0, nullptr, nullptr, a.q,
             (float*)a.scale, a.deq, a.status);
     else
         cast_tensor_kernel<FMT, DEQ, SRC_RING><<<grid, QT, 0, st>>>(
@@ -775,6 +814,66 @@ cudaError_t launch_quantize_tensor(const QuantArgs& a, cudaStream_t st) {
         else     launch_cast_tensor<FP8_E5M2, false>(a, src, grid, npart, a.hist_ring, a.hist_len, slot, a.hist_pending, a.hist_ticket, nrows, nvec, a.ld, st);
     }
     return cudaGetLastError();
+}
+
+// fp8_amax: one CTA folds the phase-1 partials into the fp32 amax.
+__global__ void __launch_bounds__(QT) amax_finalize_kernel(const uint32_t* __restrict__ partials, int32_t n,
+                                                           float* __restrict__ out, int32_t* status) {
+    __shared__ uint32_t red[32];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < n; i += QT) m = max(m, partials[i]);
+    m = block_max_u32(m, red);
+    if (threadIdx.x == 0) {
+        if (m >= 0x7F80u) report_status(status, FP8_ERR_NONFINITE);
+        *out = bf16bits_to_float(m);
+    }
+}
+
+cudaError_t launch_amax(const QuantArgs& a, float* out, cudaStream_t st) {
+    if (a.rows == 0 || a.cols == 0) return cudaMemsetAsync(out, 0, sizeof(float), st);
+    int32_t npart;
+    if (a.ld == a.cols) {
+        RQParams p{};
+        p.x = a.x;
+        p.n = a.rows * a.cols;
+        p.partials = a.partials;
+        const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rq_grid_cap(), (p.n / VEC + QT - 1) / QT));
+        rq_amax_kernel<8><<<(unsigned)grid, QT, 0, st>>>(p);
+        npart = (int32_t)grid;
+    } else {
+        const dim3 grid = tensor_grid(a.rows, a.cols / VEC);
+        amax_partials_kernel<<<grid, QT, 0, st>>>(a.x, a.rows, a.cols / VEC, a.ld, a.partials);
+        npart = (int32_t)(grid.x * grid.y);
+    }
+    amax_finalize_kernel<<<1, QT, 0, st>>>(a.partials, npart, out, a.status);
+    return cudaGetLastError();
+}
+
+template <int FMT, bool DEQ>
+static cudaError_t quantize_given_t(const QuantArgs& a, cudaStream_t st) {
+    if (a.ld == a.cols || a.rows == 0 || a.cols == 0) {
+        RQParams p{};
+        p.x = a.x;
+        p.n = a.rows * a.cols;
+        p.q = a.q;
+        p.scale = a.scale;
+        p.deq = a.deq;
+        p.status = a.status;
+        p.amax_in = a.amax_in;
+        const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rq_grid_cap(), (p.n / VEC + QT - 1) / QT));
+        rq_tensor_kernel<FMT, DEQ, RQ_GIVEN, 4><<<(unsigned)grid, QT, 0, st>>>(p);
+        return cudaGetLastError();
+    }
+    const dim3 grid = tensor_grid(a.rows, a.cols / VEC);
+    launch_cast_tensor<FMT, DEQ>(a, SRC_GIVEN, grid, 0, nullptr, 0, 0, nullptr, nullptr, a.rows, a.cols / VEC, a.ld,
+                                 st);
+    return cudaGetLastError();
+}
+
+// Per-tensor cast with a caller's amax (empty tensors still write the scale).
+cudaError_t launch_quantize_given(const QuantArgs& a, cudaStream_t st) {
+    if (a.fmt == FP8_E4M3) return a.deq ? quantize_given_t<FP8_E4M3, true>(a, st) : quantize_given_t<FP8_E4M3, false>(a, st);
+    return a.deq ? quantize_given_t<FP8_E5M2, true>(a, st) : quantize_given_t<FP8_E5M2, false>(a, st);
 }
 
 template <int FMT, bool DEQ, int G, int U, bool MX>

@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define FP8_ABI_VERSION 1
+#define FP8_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define FP8_API __attribute__((visibility("default")))
@@ -186,6 +186,93 @@ FP8_API int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int6
                            const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
                            int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy,
                            int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream);
+
+/*
+ * fp8_amax -- a_max = max |x| over a bf16 tensor, written as one fp32 to amax_dev
+ * ([FFS] section "Scale 怎样把 Tensor 塞进 E4M3": a_max = max|X|).  Exact: the
+ * largest bf16 magnitude is itself representable in fp32, and a maximum does not
+ * depend on the reduction order.
+ *   x_dev, rows, cols, ld  as for fp8_quantize (cols % 16 == 0, ld % 8 == 0,
+ *                16-byte aligned); an empty tensor gives 0.
+ *   amax_dev     device float, overwritten (needs no initialisation).
+ *   dev_status   nullable; FP8_ERR_NONFINITE for a NaN/Inf element (amax_dev is
+ *                then unspecified).
+ *   workspace_dev, ws_bytes  fp8_workspace_size(0, rows, 0, cols, FP8_SCALE_TENSOR).
+ * Together with fp8_quantize_with_amax this splits per-tensor current scaling at
+ * its one global step, the amax reduction, so that a caller can combine maxima
+ * from several places before the cast: shards of one tensor on several GPUs
+ * (an all-reduce with MAX makes every shard use the scale of the whole tensor,
+ * [FFS] section "Current Scaling": ranks synchronise so that all shards share
+ * one scale), or the amax that a GEMM epilogue already produced (fp8_epilogue_t).
+ */
+FP8_API int32_t fp8_amax(const void* x_dev, int64_t rows, int64_t cols, int64_t ld, float* amax_dev,
+                         int32_t* dev_status, void* workspace_dev, size_t ws_bytes, void* stream);
+
+/*
+ * fp8_quantize_with_amax -- the cast phase of per-tensor current scaling with a
+ * given a_max: s = fp32(max(*amax_dev, 1e-12f) / F_max), q = RNE(clip(x / s,
+ * +-F_max)), scale_dev[0] = s ([FFS] section "Scale 怎样把 Tensor 塞进 E4M3").
+ * With *amax_dev = max|x| the codes, scale and dequant equal those of
+ * fp8_quantize(..., FP8_SCALE_TENSOR, ...) bit for bit; a smaller a_max
+ * saturates the elements beyond it to +-F_max.
+ *   amax_dev     device float >= 0 read on the device (a NaN/Inf value sets
+ *                FP8_ERR_NONFINITE; the outputs are then unspecified).
+ *   q_dev, scale_dev (float[1]), dequant_dev (nullable), dev_status: as fp8_quantize.
+ *   No workspace.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ */
+FP8_API int32_t fp8_quantize_with_amax(const void* x_dev, int64_t rows, int64_t cols, int64_t ld, int32_t fmt,
+                                       const float* amax_dev, uint8_t* q_dev, float* scale_dev, void* dequant_dev,
+                                       int32_t* dev_status, void* stream);
+
+/*
+ * Epilogue options of fp8_scaled_gemm_ex / fp8_linear_forward_ex ([FFS] section
+ * "一次 FP8 GEMM 的完整精度契约": the output dtype, the output scale /
+ * requantisation when the next operator consumes FP8, and the bias fusion are
+ * part of the GEMM's contract; when the next layer runs in FP8 the epilogue can
+ * apply the output scale itself instead of writing BF16 and launching a separate
+ * cast.  [PQG] code fp8_gemm_forward takes an optional bias).  Per output element,
+ * with v the fp32 scaled accumulator of fp8_scaled_gemm:
+ *   v' = fp32(v + bias[n])                      (bias_dev != NULL; else v' = v)
+ *   y  = bf16_RNE(v')                           stored to y_dev unless y_dev is NULL
+ *   amax_dev <- max(amax_dev, |y|)              (amax_dev != NULL)
+ *   yq = RNE(clip(fp32(y) / s_y, +-F_max))      (yq_dev != NULL; s_y = *yq_scale_dev)
+ * so that yq, amax and y are exactly what "store Y in bf16, then reduce its amax /
+ * cast it with scale s_y" would give.
+ *   bias_dev      nullable bf16 [N], 16-byte aligned.
+ *   amax_dev      nullable device float holding a value >= 0 before the call (e.g. 0);
+ *                 the maximum |y| over the output is folded in with an atomic max.
+ *   yq_dev        nullable uint8 [M, ldq] codes of format yq_fmt (E4M3 or E5M2).
+ *   yq_scale_dev  device float s_y, the dequantisation multiplier of yq, required
+ *                 with yq_dev; a value that is not a positive normal fp32 with a
+ *                 finite reciprocal sets FP8_ERR_INVALID_ARG in dev_status (codes
+ *                 then unspecified).
+ *   ldq           row stride of yq in bytes, >= N.
+ * A NULL fp8_epilogue_t pointer, or one with every pointer NULL, is plain
+ * fp8_scaled_gemm.  With yq_dev set, y_dev may be NULL (FP8 output only).
+ */
+typedef struct {
+    const void* bias_dev;
+    float* amax_dev;
+    uint8_t* yq_dev;
+    const float* yq_scale_dev;
+    int32_t yq_fmt;
+    int64_t ldq;
+} fp8_epilogue_t;
+
+/* fp8_scaled_gemm with the epilogue options above (epi nullable). */
+FP8_API int32_t fp8_scaled_gemm_ex(const uint8_t* a_dev, const void* a_scale_dev, int32_t a_mode, int32_t fmt_a,
+                                   const uint8_t* b_dev, const void* b_scale_dev, int32_t b_mode, int32_t fmt_b,
+                                   int64_t M, int64_t N, int64_t K, void* y_dev, int64_t ldy,
+                                   const fp8_epilogue_t* epi, int32_t* dev_status, void* workspace_dev,
+                                   size_t ws_bytes, void* stream);
+
+/* fp8_linear_forward with the epilogue options above (epi nullable). */
+FP8_API int32_t fp8_linear_forward_ex(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt,
+                                      int32_t x_mode, fp8_history_t* hist,
+                                      const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
+                                      int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy,
+                                      const fp8_epilogue_t* epi, int32_t* dev_status,
+                                      void* workspace_dev, size_t ws_bytes, void* stream);
 
 /*
  * fp8_linear_forward_noalloc -- fp8_linear_forward for callers that cannot

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_status_strings(lib):
     from fp8_dynamic_scaled_b200 import binding as b
-    assert b.fp8_abi_version() == 1
+    assert b.fp8_abi_version() == 2
     assert b.fp8_status_string(0) == "FP8_OK"
     assert b.fp8_status_string(5) == "FP8_ERR_TIMEOUT"
     assert b.fp8_status_string(99) == "FP8_ERR_UNKNOWN"
