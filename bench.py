@@ -76,7 +76,7 @@ def load_peaks():
 
 def source_digest():
     h = hashlib.sha256()
-    for fn in ("gemm_sm100.cu", "quantize.cu", "ptx.cuh", "common.cuh"):
+    for fn in ("gemm_sm100.cu", "gemm_common.cuh", "decode_sm100.cu", "quantize.cu", "ptx.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "fp8_dynamic_scaled_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
