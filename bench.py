@@ -40,6 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 WORKLOADS = {
     "llama70b_prefill": dict(M=4096, K=8192, N=28672, x_mode=1, w_mode=1),
+    # the same layer at decode: 16 tokens per call (the weight-streaming kernel)
+    "llama70b_decode": dict(M=16, K=8192, N=28672, x_mode=1, w_mode=1),
     "block_scaled": dict(M=8192, K=8192, N=28672, x_mode=2, w_mode=3),
     "mx": dict(M=16384, K=8192, N=8192, x_mode=4, w_mode=4),
 }
@@ -157,7 +159,7 @@ def make_workload(torch, fp8, name, rank):
     from fp8_dynamic_scaled_b200 import inputs
     wl = WORKLOADS[name]
     M, K, N = wl["M"], wl["K"], wl["N"]
-    if name == "llama70b_prefill":
+    if name in ("llama70b_prefill", "llama70b_decode"):
         x, w = inputs.llama70b_prefill(M, K, N)
     elif name == "block_scaled":
         x, w = inputs.block_scaled(M, K, N)
@@ -703,13 +705,23 @@ def main():
                      "kernel": "fp8_gemm_pair_kernel" if variant == "ROWSCALE" and M >= 256 else f"fp8_gemm_kernel<{variant}>",
                      "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16} (fp8/bf16 nominal ratio)",
                      "gemm_us_avg": g_avg * 1e3},
+    }
+    if variant == "ROWSCALE" and M <= 64:
+        # few tokens: the GEMM is bound by streaming W (and X, scales, Y) from HBM
+        gbytes = N * K + M * K + 4 * (M + N) + 2 * M * N
+        line["roofline"] = {"bound": "hbm", "achieved": gbytes / (g_avg * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                            "unit": "GB/s", "frac": gbytes / (g_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                            "traffic": profiled_traffic(f"gemm_decode_{args.workload}"), "kernel": "fp8_decode_kernel",
+                            "peak_source": f"{peak_src} hbm_gbs", "gemm_us_avg": g_avg * 1e3,
+                            "algorithmic_bytes": gbytes, "gemm_tflops": gemm_tflops}
+    line.update({
         "quantize": {"kernel": qkernel, "us_avg": q_avg * 1e3, "algorithmic_bytes": xbytes,
                      "GB_per_s": xbytes / (q_avg * 1e-3) / 1e9,
                      "frac_of_hbm": xbytes / (q_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "share_of_gemm_time": q_avg / g_avg},
         "clocks": clocks,
         "gpu_launches": args.steps * (quantize_launches(wl["x_mode"]) + 1),
-    }
+    })
     if rank == 0:
         e2e_ms, h2d, d2h = time_e2e(torch, fp8, wl, max(3, min(args.steps, 10)), 2, stream)
         line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
