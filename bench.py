@@ -456,6 +456,41 @@ def extras(torch, fp8, stream, peaks):
                              "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
                              "tflops": 2.0 * Md * N * K / (ms * 1e-3) / 1e12}
         res["note"] = "N=28672, K=8192 per-row scales; bytes = W codes + X codes + scales + bf16 Y"
+        # the whole decode layer: fp8_linear_forward (X quantize, then the GEMM launched as
+        # its programmatic dependent, streaming W while X is quantised) against the same
+        # two steps as separate calls; interleaved rounds of 50 calls, median round
+        xh_all = inputs.llama70b_prefill(64, K, N, with_w=False)[0]
+        for Md in (1, 16, 64):
+            xd = to_dev_bf16(torch, xh_all[:Md])
+            yd = torch.empty((Md, N), dtype=torch.bfloat16, device="cuda")
+            lws = fp8.workspace_for(2, Md, N, K, fp8.FP8_SCALE_ROW)
+            xq_d, xs_d, _ = fp8.empty_quant_outputs(Md, K, fp8.FP8_SCALE_ROW)
+            qws = fp8.workspace_for(0, Md, 0, K, fp8.FP8_SCALE_ROW)
+            fns = {
+                "linear_forward": lambda: fp8.fp8_linear_forward(xd, fp8.FP8_E4M3, fp8.FP8_SCALE_ROW, wq, wsc,
+                                                                 fp8.FP8_SCALE_ROW, fp8.FP8_E4M3, yd, lws,
+                                                                 stream=stream),
+                "quantize_then_gemm": lambda: (
+                    fp8.fp8_quantize(xd, fp8.FP8_E4M3, fp8.FP8_SCALE_ROW, xq_d, xs_d, workspace=qws, stream=stream),
+                    fp8.fp8_scaled_gemm(xq_d, xs_d, fp8.FP8_SCALE_ROW, fp8.FP8_E4M3, wq, wsc, fp8.FP8_SCALE_ROW,
+                                        fp8.FP8_E4M3, yd, stream=stream)),
+            }
+            per = {k: [] for k in fns}
+            with torch.cuda.stream(stream):
+                for f in fns.values():
+                    f()
+            torch.cuda.synchronize()
+            for _ in range(5):
+                for k, f in fns.items():
+                    with torch.cuda.stream(stream):
+                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record(stream)
+                        for _ in range(50):
+                            f()
+                        b.record(stream)
+                    torch.cuda.synchronize()
+                    per[k].append(a.elapsed_time(b) / 50 * 1e3)
+            res[f"layer_M{Md}_us"] = {k: statistics.median(v) for k, v in per.items()}
         out["decode_shapes"] = res
     except Exception as ex:
         out["decode_shapes"] = {"error": str(ex)[:200]}

@@ -155,7 +155,7 @@ int32_t check_gemm_args(const uint8_t* a, const void* sa, int32_t am, int32_t fa
 
 int32_t gemm_impl(const uint8_t* a, const void* sa, int32_t am, int32_t fa, const uint8_t* b, const void* sb,
                   int32_t bm, int32_t fb, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int32_t* status,
-                  cudaStream_t st, const fp8_epilogue_t* epi = nullptr) {
+                  cudaStream_t st, const fp8_epilogue_t* epi = nullptr, bool a_just_quantized = false) {
     if (M == 0 || N == 0) return FP8_OK;
     const bool ext = epi_active(epi);
     if (K == 0 && !ext) return cuda_status(launch_zero_output(static_cast<uint16_t*>(y), M, N, ldy, st));
@@ -182,6 +182,7 @@ int32_t gemm_impl(const uint8_t* a, const void* sa, int32_t am, int32_t fa, cons
     g.y = static_cast<uint16_t*>(y);
     g.ldy = ldy;
     g.status = status;
+    g.a_from_previous_kernel = a_just_quantized;
     if (K == 0) return cuda_status(launch_zero_k_epilogue(g, st));
     return cuda_status(launch_gemm(g, st));
 }
@@ -324,7 +325,9 @@ int32_t fp8_linear_forward_ex(const void* x_dev, int64_t M, int64_t K, int64_t l
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = quantize_impl(x_dev, M, K, ldx, x_fmt, x_mode, xq, xs, hist, nullptr, dev_status, part, partials_bytes(), st);
     if (rc != FP8_OK) return rc;
-    return gemm_impl(xq, xs, gm_a, x_fmt, w_dev, w_scale_dev, w_mode, w_fmt, M, N, K, y_dev, ldy, dev_status, st, epi);
+    // the quantize kernel just enqueued wrote X's codes and scales and nothing else
+    return gemm_impl(xq, xs, gm_a, x_fmt, w_dev, w_scale_dev, w_mode, w_fmt, M, N, K, y_dev, ldy, dev_status, st, epi,
+                     /*a_just_quantized=*/true);
 }
 
 int32_t fp8_linear_forward(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt, int32_t x_mode,

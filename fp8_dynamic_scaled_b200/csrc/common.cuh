@@ -124,6 +124,16 @@ __device__ __forceinline__ void st_v4_stream(void* p, uint4 v) {
     __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
+// Programmatic dependent launch: let the next kernel in the stream (if it was
+// launched as a programmatic dependent) start now; it waits for this grid's results
+// with pdl_wait() before it reads them.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the preceding grid (if this one was launched as its programmatic
+// dependent) has completed and its writes are visible; a no-op otherwise.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Record the first device-side error in a caller-owned status word.
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
     if (status) atomicCAS(status, 0, code);

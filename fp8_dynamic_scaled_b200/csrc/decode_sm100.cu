@@ -121,17 +121,20 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
+        // Step i of this CTA is K stage i % nkc of chunk i / nkc.  When the kernel runs
+        // as the programmatic dependent of the kernel that quantised X (p.pdl), W cannot
+        // be that kernel's output: the first ring of W loads goes out at once, and only
+        // the X loads wait for the quantiser's results (pdl_wait).
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0;
-            bool ok = true;
-            for (int32_t j = 0; j < range.nch && ok; ++j) {
+            const int32_t total = range.nch * nkc;
+            const int32_t pre = p.pdl ? min(S, total) : 0;
+            auto issue = [&](int32_t i, uint32_t stage, bool w_part, bool x_part) {
                 int32_t n0, w;
-                decode_chunk(range, j, n0, w);
-                for (int32_t kc = 0; kc < nkc; ++kc) {
-                    const int32_t kb0 = kc * d.kbs;
-                    const int32_t kbs = min(d.kbs, p.num_kb - kb0);
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-                    uint8_t* st = stages + stage * d.stage_bytes;
+                decode_chunk(range, i / nkc, n0, w);
+                const int32_t kb0 = (i % nkc) * d.kbs;
+                const int32_t kbs = min(d.kbs, p.num_kb - kb0);
+                uint8_t* st = stages + stage * d.stage_bytes;
+                if (w_part) {
                     ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)kbs * (uint32_t)(w + d.nt) * BK);
                     // row group by row group, each group's K blocks back to back
                     for (int32_t r = 0; r < w;) {
@@ -141,10 +144,19 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                                              (kb0 + b) * BK, n0 + r);
                         r += big ? 64 : D_UNIT;
                     }
+                }
+                if (x_part)
                     for (int32_t b = 0; b < kbs; ++b)
                         ptx::tma_load_2d(st + x_off + b * d.nt * BK, &tmX, &full[stage], (kb0 + b) * BK, 0);
-                    if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
-                }
+            };
+            for (int32_t i = 0; i < pre; ++i) issue(i, (uint32_t)i, true, false);   // fresh ring: no waits
+            pdl_wait();
+            for (int32_t i = 0; i < pre; ++i) issue(i, (uint32_t)i, false, true);
+            uint32_t stage = (uint32_t)(pre % S), phase = (pre == S) ? 1u : 0u;
+            for (int32_t i = pre; i < total; ++i) {
+                if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) break;
+                issue(i, stage, true, true);
+                if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
             }
         }
     } else if (warp == 1) {
@@ -187,6 +199,7 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue: lane = weight row
+        pdl_wait();                           // X's scales (and epilogue inputs) may be just written
         const int quarter = warp & 3;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         uint32_t amax_bits = 0;               // |y| as fp32 patterns (order-preserving for y >= 0)
@@ -282,7 +295,18 @@ static cudaError_t launch_decode_t(const GemmArgs& g, GemmParams p, cudaStream_t
     p.idesc = (1u << 4) | ((uint32_t)g.fmt_b << 7) | ((uint32_t)g.fmt_a << 10) | ((uint32_t)(d.nt >> 3) << 17) |
               ((uint32_t)(D_TILE >> 4) << 24);
     const int grid = std::max(1, std::min(d.units, num_sms()));
-    fp8_decode_kernel<EXT><<<grid, 192, D_SMEM, st>>>(tx, t64, t16, p, d);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = D_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_decode_kernel<EXT>, tx, t64, t16, p, d);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -53,6 +53,8 @@ struct GemmParams {
     int64_t ldq;
     int32_t yq_fmt;
     int32_t yq_vec;         // yq rows start 16-byte aligned
+    // launched as the programmatic dependent of the kernel that produced A (and only A)
+    int32_t pdl;
 };
 
 // ---------------------------------------------------------------- bounded waits

@@ -842,7 +842,10 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
         p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
         // a few tokens: stream W across all SMs; CTA pairs once M spans a 256-row tile;
         // a single CTA per tile in between
-        if (g.M <= D_MAX_TOKENS) return launch_decode(g, p, st);
+        if (g.M <= D_MAX_TOKENS) {
+            p.pdl = g.a_from_previous_kernel ? 1 : 0;
+            return launch_decode(g, p, st);
+        }
         if (g.M >= P_BM) return p.ext ? launch_pair<true>(g, p, st) : launch_pair<false>(g, p, st);
         return p.ext ? launch_variant<V_ROWSCALE, true>(g, p, st) : launch_variant<V_ROWSCALE, false>(g, p, st);
     }

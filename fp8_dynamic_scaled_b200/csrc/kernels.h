@@ -53,6 +53,9 @@ struct GemmArgs {
     const float* yq_scale;   // s_y
     int32_t yq_fmt;
     int64_t ldq;
+    // the kernel just before the GEMM on the stream wrote A and its scales and nothing
+    // else: the GEMM may start on B before A is ready (programmatic dependent launch)
+    bool a_from_previous_kernel;
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);

@@ -122,6 +122,7 @@ __device__ __forceinline__ float given_amax(const float* a, int32_t* status) {
 __global__ void __launch_bounds__(QT) amax_partials_kernel(const uint16_t* __restrict__ x, int64_t nrows,
                                                            int64_t nvec, int64_t ld,
                                                            uint32_t* __restrict__ partials) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     uint32_t m2 = 0;
     const int64_t stride = (int64_t)gridDim.x * QT;
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
     float* ring, int32_t ring_len, int32_t slot, float* pending, uint32_t* ticket,
     uint8_t* __restrict__ q, float* __restrict__ scale_out, uint16_t* __restrict__ deq,
     int32_t* status) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     // ---- the scale
     uint32_t src = 0;
@@ -250,6 +252,7 @@ __global__ void __launch_bounds__(QT) quant_segment_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     int32_t seg_vec, int64_t nseg_per_row, int64_t nseg,
     uint8_t* __restrict__ q, void* __restrict__ scale, uint16_t* __restrict__ deq, int32_t* status) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     const int lane_g = threadIdx.x & (G - 1);
     const int64_t group = ((int64_t)blockIdx.x * QT + threadIdx.x) / G;
     const int64_t ngroups = (int64_t)gridDim.x * (QT / G);
@@ -321,6 +324,7 @@ __global__ void __launch_bounds__(QT) quant_row_kernel(const uint16_t* __restric
                                                        int64_t cols, int64_t ld, uint8_t* __restrict__ q,
                                                        float* __restrict__ scale, uint16_t* __restrict__ deq,
                                                        int32_t* status) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     const int64_t nvec = cols / VEC;
     for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
@@ -371,6 +375,7 @@ __global__ void __launch_bounds__(QT) quant_block128_kernel(const uint16_t* __re
                                                             int64_t cols, int64_t ld, uint8_t* __restrict__ q,
                                                             float* __restrict__ scale, uint16_t* __restrict__ deq,
                                                             int32_t* status) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     constexpr int UB = 128 * 16 / QT;   // 8 vectors per thread
     const int64_t ncb = (cols + 127) / 128;
@@ -540,6 +545,7 @@ struct RQParams {
 // One CTA per row; the row (<= QT * VPT vectors) is held in registers.
 template <int FMT, bool DEQ, int VPT, int MINB>
 __global__ void __launch_bounds__(QT, MINB) rq_row_kernel(const RQParams p) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     const int64_t r = blockIdx.x;
     const uint16_t* src = p.x + r * p.ld;
@@ -576,6 +582,7 @@ __global__ void __launch_bounds__(QT, MINB) rq_row_kernel(const RQParams p) {
 // for a fixed j the vectors of one block sit in G consecutive lanes.
 template <int FMT, bool DEQ, int KIND, int VPT>
 __global__ void __launch_bounds__(QT, 8) rq_block_kernel(const RQParams p) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     constexpr int G = KIND == RQ_B128 ? 16 : 4;
     const int64_t e0 = (int64_t)blockIdx.x * QT * VPT * VEC;
     uint4 v[VPT];
@@ -617,6 +624,7 @@ __global__ void __launch_bounds__(QT, 8) rq_block_kernel(const RQParams p) {
 // Per-tensor phase 1: U independent loads in flight per thread.
 template <int U>
 __global__ void __launch_bounds__(QT, 8) rq_amax_kernel(const RQParams p) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     const int64_t nvec = p.n / VEC;
     uint32_t m2 = 0;
@@ -639,6 +647,7 @@ __global__ void __launch_bounds__(QT, 8) rq_amax_kernel(const RQParams p) {
 // leave them 48 registers.)
 template <int FMT, bool DEQ, int KIND, int U>
 __global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(const RQParams p) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
     __shared__ uint32_t red[32];
     uint32_t src = 0;
     if (KIND == RQ_CAST) {
