@@ -14,7 +14,7 @@
 //     of 16 rows, as evenly as the units allow, and each range is done in chunks of
 //     at most 128 rows.  Rows of the 128-row tile past a chunk are not loaded; their
 //     accumulator lanes are never read.  No partial sums cross CTAs;
-//   - HBM is read in long runs: a stage holds KBS (4, or 2 with more tokens) K blocks
+//   - HBM is read in long runs: a stage holds KBS (4, or 3 with more tokens) K blocks
 //     of 128 bytes of the chunk, loaded as 64-row (and 16-row) TMA boxes issued
 //     row-group by row-group, so each row's KBS consecutive blocks are requested back
 //     to back.  (Measured on this part with loads alone: 128-row x 128-byte boxes
@@ -38,7 +38,7 @@ constexpr int D_MAX_KBS = 4;
 constexpr int D_MAX_STAGES = 8;
 constexpr uint32_t D_TILE_BYTES = D_TILE * BK;          // 16 KB: one K block of a chunk
 constexpr uint32_t D_BAR_BYTES = 1024;                  // barriers + misc, ahead of the stages
-constexpr uint32_t D_SMEM = 227 * 1024;                 // dynamic shared memory requested
+constexpr uint32_t D_SMEM = 227 * 1024;                 // dynamic shared memory budget
 
 struct DecodeParams {
     int32_t units;         // ceil(N / 16)
@@ -272,7 +272,9 @@ static cudaError_t launch_decode_t(const GemmArgs& g, GemmParams p, cudaStream_t
     DecodeParams d{};
     d.nt = (int32_t)((g.M + 15) / 16 * 16);
     d.units = (int32_t)((g.N + D_UNIT - 1) / D_UNIT);
-    d.kbs = d.nt <= 16 ? D_MAX_KBS : 2;
+    // 4 K blocks per stage (3 stages) up to 16 tokens; with more tokens the X tiles grow
+    // and 3 blocks (3 stages) beat both 4 blocks (2 stages) and 2 blocks (5 stages)
+    d.kbs = d.nt <= 16 ? D_MAX_KBS : 3;
     d.stage_bytes = (uint32_t)d.kbs * (D_TILE_BYTES + (uint32_t)d.nt * BK);
     d.stages = (int32_t)std::min<uint32_t>(D_MAX_STAGES, (D_SMEM - 1024 - D_BAR_BYTES) / d.stage_bytes);
     CUtensorMap tx, t64, t16;
@@ -290,6 +292,9 @@ static cudaError_t launch_decode_t(const GemmArgs& g, GemmParams p, cudaStream_t
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
+    // request only what the stages use, so that a small kernel running just before (the
+    // X quantize, whose dependent this kernel may be) can share an SM with this one
+    const uint32_t smem = 1024 + D_BAR_BYTES + (uint32_t)d.stages * d.stage_bytes;
     // swapped operands: the instruction's A is W (format fmt_b), its B is X (fmt_a);
     // M = 128 weight rows, N = nt tokens
     p.idesc = (1u << 4) | ((uint32_t)g.fmt_b << 7) | ((uint32_t)g.fmt_a << 10) | ((uint32_t)(d.nt >> 3) << 17) |
@@ -298,7 +303,7 @@ static cudaError_t launch_decode_t(const GemmArgs& g, GemmParams p, cudaStream_t
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(192);
-    cfg.dynamicSmemBytes = D_SMEM;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
