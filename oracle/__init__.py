@@ -277,6 +277,25 @@ def epilogue_ref(y_ref, bound, bias_bf16=None):
     return y_ref + b, bound + np.abs(b)
 
 
+def weight_only_ref(x_bf16, w_codes, w_scale, w_mode: int, w_fmt: int):
+    """Weight-only FP8 linear ([FFS] "FP8 formats, scaling and LLM inference", section
+    "Weight-only FP8 与 W8A8 FP8": the weight is stored in FP8, the activation stays
+    BF16): y[m, n] = sum_k x[m, k] * (s_w[n] * decode(w[n, k])) in fp64, with the
+    bound sum_k |same product| of the acceptance rule.  s_w is the per-tensor or
+    per-row scale of the weight's quantisation (the matmul is a library step)."""
+    x = bf16_to_f32(np.asarray(x_bf16, np.uint16)).astype(np.float64)
+    table = decode_table(w_fmt)
+    wd = table[np.asarray(w_codes, np.uint8)]
+    s = np.asarray(w_scale, np.float64).reshape(-1)
+    if w_mode == ROW:
+        wd = wd * s[:, None]
+    elif w_mode in (TENSOR, DELAYED):
+        wd = wd * s[0]
+    else:
+        raise ValueError("weight-only takes per-tensor or per-row weight scales")
+    return x @ wd.T, np.abs(x) @ np.abs(wd).T
+
+
 def requant_interval(y_ref, lim, s_y: float, fmt: int):
     """Values an FP8 output code may decode to when the bf16 output y lies within
     [y_ref - lim, y_ref + lim] and is then quantised with the fixed scale s_y

@@ -135,3 +135,34 @@ def test_requant_interval_brackets_every_value_in_range(fmt):
         c = table[oracle.quant_scaled(v, s, fmt)]
         assert np.all((c[inside] >= lo[inside]) & (c[inside] <= hi[inside]))
     assert np.all(lo <= hi)
+
+
+# ------------------------------------------------------------ weight-only reference
+def test_weight_only_exact_integer():
+    """Integer activations (exact in bf16), small-integer codes, unit scale: an int64 matmul."""
+    g = np.random.default_rng(51)
+    M, N, K = 5, 40, 96
+    x_int = g.integers(-20, 21, (M, K))
+    w_int = g.integers(-6, 7, (N, K))
+    codes = _codes_of(w_int, E4M3)
+    y, bound = oracle.weight_only_ref(inputs.bf16_bits(x_int.astype(np.float32)), codes, np.ones(1, np.float32),
+                                      oracle.TENSOR, E4M3)
+    assert np.array_equal(y, (x_int @ w_int.T).astype(np.float64))
+    assert np.array_equal(bound, (np.abs(x_int) @ np.abs(w_int).T).astype(np.float64))
+
+
+def test_weight_only_identity_and_row_scales():
+    """W = identity codes with per-row scales s: y[m, n] = x[m, n] * s[n]; and the per-row
+    reference equals a per-tensor one when every row has the same scale."""
+    g = np.random.default_rng(52)
+    K = 64
+    x = inputs.bf16_bits(g.standard_normal((3, K)).astype(np.float32))
+    eye = _codes_of(np.eye(K), E5M2)
+    s = (np.arange(1, K + 1) / 8.0).astype(np.float32)
+    y, _ = oracle.weight_only_ref(x, eye, s, oracle.ROW, E5M2)
+    assert np.array_equal(y, oracle.bf16_to_f32(x).astype(np.float64) * s.astype(np.float64)[None, :])
+    w = g.integers(0, 256, (7, K)).astype(np.uint8)
+    w[(w & 0x7F) == 0x7F] = 0          # keep E4M3 codes finite
+    y1, _ = oracle.weight_only_ref(x, w, np.full(7, 0.25, np.float32), oracle.ROW, E4M3)
+    y2, _ = oracle.weight_only_ref(x, w, np.array([0.25], np.float32), oracle.TENSOR, E4M3)
+    assert np.array_equal(y1, y2)
