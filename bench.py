@@ -511,6 +511,15 @@ def extras(torch, fp8, stream, peaks):
                     torch.cuda.synchronize()
                     per[k].append(a.elapsed_time(b) / 50 * 1e3)
             res[f"layer_M{Md}_us"] = {k: statistics.median(v) for k, v in per.items()}
+        # weight-only FP8 (X stays bf16, W codes converted on chip): the same layer
+        for Md in (1, 16, 64):
+            xd = to_dev_bf16(torch, xh_all[:Md])
+            yd = torch.empty((Md, N), dtype=torch.bfloat16, device="cuda")
+            med, _ = time_kernel(torch, lambda: fp8.fp8_weight_only_linear(xd, wq, wsc, fp8.FP8_SCALE_ROW, fp8.FP8_E4M3,
+                                                                           yd, stream=stream), 50, stream)
+            nbytes = N * K + 2 * Md * K + 4 * N + 2 * Md * N
+            res[f"weight_only_M{Md}"] = {"us": med * 1e3, "GB_per_s": nbytes / (med * 1e-3) / 1e9,
+                                         "frac_of_hbm": nbytes / (med * 1e-3) / 1e9 / hbm}
         out["decode_shapes"] = res
     except Exception as ex:
         out["decode_shapes"] = {"error": str(ex)[:200]}

@@ -14,7 +14,7 @@ import importlib
 
 __all__ = ["fp8_abi_version", "fp8_status_string", "fp8_device_check", "fp8_workspace_size", "fp8_quantize",
            "fp8_scaled_gemm", "fp8_linear_forward", "fp8_amax", "fp8_quantize_with_amax", "fp8_scaled_gemm_ex",
-           "fp8_linear_forward_ex", "History", "FP8Error", "binding", "inputs"]
+           "fp8_linear_forward_ex", "fp8_weight_only_linear", "History", "FP8Error", "binding", "inputs"]
 
 
 def __getattr__(name):

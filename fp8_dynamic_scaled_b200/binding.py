@@ -31,7 +31,9 @@ FP8_ERR_NONFINITE, FP8_ERR_TIMEOUT, FP8_ERR_CUDA, FP8_ERR_WORKSPACE = 4, 5, 6, 7
 
 EXPORTED = ("fp8_abi_version", "fp8_status_string", "fp8_device_check", "fp8_workspace_size",
             "fp8_quantize", "fp8_scaled_gemm", "fp8_linear_forward", "fp8_linear_forward_noalloc",
-            "fp8_amax", "fp8_quantize_with_amax", "fp8_scaled_gemm_ex", "fp8_linear_forward_ex")
+            "fp8_amax", "fp8_quantize_with_amax", "fp8_scaled_gemm_ex", "fp8_linear_forward_ex",
+            "fp8_weight_only_linear")
+FP8_WEIGHT_ONLY_MAX_TOKENS = 64
 FP8_NOALLOC_SCRATCH_BYTES = 4194304
 
 
@@ -71,6 +73,8 @@ _lib.fp8_linear_forward_ex.restype = _I32
 _lib.fp8_linear_forward_ex.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P, _P,
                                        _I32, _I32, _I64, _P, _I64, ctypes.POINTER(fp8_epilogue_t), _P, _P, _SZ,
                                        _P]
+_lib.fp8_weight_only_linear.restype = _I32
+_lib.fp8_weight_only_linear.argtypes = [_P, _I64, _I64, _I64, _P, _P, _I32, _I32, _I64, _P, _I64, _P, _P]
 _lib.fp8_linear_forward_noalloc.restype = _I32
 _lib.fp8_linear_forward_noalloc.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P,
                                             _P, _I32, _I32, _I64, _P, _I64, _P, _P]
@@ -252,6 +256,19 @@ def fp8_linear_forward_ex(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, worksp
                                     w_mode, w_fmt, N, _ptr(y), ldy, ctypes.byref(epi) if epi is not None else None,
                                     _ptr(dev_status), _ptr(workspace), _nbytes(workspace), _stream(stream))
     _check(rc, "fp8_linear_forward_ex")
+
+
+def fp8_weight_only_linear(x, w, w_scale, w_mode, w_fmt, y, *, dev_status=None, stream=None):
+    """y [M, N] bf16 = x [M, K] bf16 times the FP8 weight w [N, K] (codes) with its scale."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.uint8 or y.dtype != torch.bfloat16:
+        raise TypeError("x bf16, w uint8 codes, y bf16")
+    M, K = x.shape
+    N = w.shape[0]
+    ldx = x.stride(0) if M > 1 else K
+    ldy = y.stride(0) if y.shape[0] > 1 else y.shape[1]
+    rc = _lib.fp8_weight_only_linear(_ptr(x), M, K, ldx, _ptr(w), _ptr(w_scale), w_mode, w_fmt, N, _ptr(y), ldy,
+                                     _ptr(dev_status), _stream(stream))
+    _check(rc, "fp8_weight_only_linear")
 
 
 def fp8_linear_forward_noalloc(x, x_fmt, x_mode, w, w_scale, w_mode, w_fmt, y, *, hist: History | None = None,

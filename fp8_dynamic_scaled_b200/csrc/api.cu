@@ -303,6 +303,43 @@ int32_t fp8_scaled_gemm_ex(const uint8_t* a_dev, const void* a_scale_dev, int32_
                      dev_status, static_cast<cudaStream_t>(stream), epi);
 }
 
+int32_t fp8_weight_only_linear(const void* x_dev, int64_t M, int64_t K, int64_t ldx, const uint8_t* w_dev,
+                               const void* w_scale_dev, int32_t w_mode, int32_t w_fmt, int64_t N, void* y_dev,
+                               int64_t ldy, int32_t* dev_status, void* stream) {
+    if (w_fmt != FP8_E4M3 && w_fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (w_mode != FP8_SCALE_TENSOR && w_mode != FP8_SCALE_ROW && w_mode != FP8_SCALE_DELAYED) return FP8_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || M > FP8_WEIGHT_ONLY_MAX_TOKENS) return FP8_ERR_INVALID_ARG;
+    if (N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return FP8_ERR_INVALID_ARG;
+    if (K % 16 != 0 || ldy < N || (K > 0 && ldx < K)) return FP8_ERR_INVALID_ARG;
+    if (M > 0 && N > 0) {
+        if (y_dev == nullptr) return FP8_ERR_INVALID_ARG;
+        if (K > 0 && (x_dev == nullptr || w_dev == nullptr || w_scale_dev == nullptr)) return FP8_ERR_INVALID_ARG;
+    }
+    // X and W are not read when K == 0
+    if (K > 0 && (ldx % 8 != 0 || !aligned16(x_dev) || !aligned16(w_dev))) return FP8_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(w_scale_dev) & 3u) != 0 || (reinterpret_cast<uintptr_t>(y_dev) & 1u) != 0)
+        return FP8_ERR_ALIGNMENT;
+    int32_t rc = device_gate();
+    if (rc != FP8_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 0 || N == 0) return FP8_OK;
+    if (K == 0) return cuda_status(launch_zero_output(static_cast<uint16_t*>(y_dev), M, N, ldy, st));
+    WoArgs g{};
+    g.x = static_cast<const uint16_t*>(x_dev);
+    g.ldx = ldx;
+    g.w = w_dev;
+    g.sw = w_scale_dev;
+    g.w_row_scales = w_mode == FP8_SCALE_ROW;
+    g.w_fmt = w_fmt;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.y = static_cast<uint16_t*>(y_dev);
+    g.ldy = ldy;
+    g.status = dev_status;
+    return cuda_status(launch_weight_only(g, st));
+}
+
 int32_t fp8_linear_forward_ex(const void* x_dev, int64_t M, int64_t K, int64_t ldx, int32_t x_fmt, int32_t x_mode,
                            fp8_history_t* hist, const uint8_t* w_dev, const void* w_scale_dev, int32_t w_mode,
                               int32_t w_fmt, int64_t N, void* y_dev, int64_t ldy, const fp8_epilogue_t* epi,

@@ -59,6 +59,20 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
+
+struct WoArgs {              // weight-only FP8 linear (wo_sm100.cu)
+    const uint16_t* x;       // bf16 [M, K], row stride ldx
+    int64_t ldx;
+    const uint8_t* w;        // FP8 codes [N, K]
+    const void* sw;          // fp32 scale: [1] or [N]
+    bool w_row_scales;
+    int32_t w_fmt;
+    int64_t M, N, K;
+    uint16_t* y;             // bf16 [M, N], row stride ldy
+    int64_t ldy;
+    int32_t* status;
+};
+cudaError_t launch_weight_only(const WoArgs& g, cudaStream_t st);
 cudaError_t launch_zero_output(uint16_t* y, int64_t M, int64_t N, int64_t ldy, cudaStream_t st);
 cudaError_t launch_zero_k_epilogue(const GemmArgs& g, cudaStream_t st);
 

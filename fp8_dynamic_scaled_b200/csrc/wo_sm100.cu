@@ -1,0 +1,337 @@
+// wo_sm100.cu -- weight-only FP8 linear for few tokens (M <= 64), sm_100a.
+//
+//   Y[m, n] = bf16( s_w[n] sum_k x[m,k] decode(w[n,k]) ),  X bf16, W FP8 codes,
+//   s_w per tensor or per output channel
+//
+// [FFS] "FP8 formats, scaling and LLM inference", section "Weight-only FP8 与 W8A8
+// FP8": the weight is stored in FP8 and the activation stays BF16; the kernel reads
+// FP8 and converts it, and the gain is the weight's memory and bandwidth.  tcgen05
+// multiplies BF16 by BF16 (kind::f16) but not BF16 by FP8, so:
+//   - the weight streams exactly as in the W8A8 decode kernel (decode_sm100.cu):
+//     one contiguous range of W rows per SM in 16-row units, chunks of <= 128 rows,
+//     stages of 3 K blocks loaded as 64-/16-row boxes issued row group by row group;
+//     every FP8 code is read from HBM once;
+//   - eight converter warps turn each 128-row x 64-element half of a K block into
+//     BF16 (exact: every E4M3 and E5M2 value is a BF16 value) and write it in the
+//     K-major 128-byte-swizzled layout the tensor core reads, into a two-slot ring;
+//   - the MMA warp issues tcgen05.mma kind::f16 with the weight as A (M = 128 rows)
+//     and the tokens as B (N = M rounded up to 16, X tiles loaded by TMA as BF16),
+//     FP32 accumulators double-buffered in TMEM across chunks;
+//   - the epilogue warp of a TMEM lane quarter owns 32 weight rows and writes
+//     bf16(acc * s_w[n]) for every token.
+// Every wait is bounded as in the other kernels.
+#include "gemm_common.cuh"
+
+namespace fp8b {
+
+constexpr int WO_UNIT = 16;                          // rows of W per work unit
+constexpr int WO_TILE = 128;                         // rows of W per MMA
+constexpr int WO_KBS = 3;                            // K blocks (128 codes) per stage
+constexpr int WO_MAX_STAGES = 4;
+constexpr int WO_SLOTS = 2;                          // BF16 weight ring
+constexpr int WO_CONV_WARPS = 8, WO_EPI_WARPS = 4;
+constexpr int WO_FIRST_CONV = 2, WO_FIRST_EPI = WO_FIRST_CONV + WO_CONV_WARPS;
+constexpr int WO_THREADS = 32 * (WO_FIRST_EPI + WO_EPI_WARPS);     // 448
+constexpr uint32_t WO_W8_BYTES = WO_TILE * BK;       // 16 KB: FP8 codes of one K block
+constexpr uint32_t WO_HALF_BYTES = WO_TILE * 128;    // 16 KB: 64 BF16 values of 128 rows
+constexpr uint32_t WO_BAR_BYTES = 1024;
+constexpr uint32_t WO_SMEM = 227 * 1024;
+
+struct WoParams {
+    int32_t units;          // ceil(N / 16)
+    int32_t nt;             // tokens per MMA: M rounded up to 16
+    int32_t stages;
+    uint32_t stage_bytes;   // WO_KBS * (WO_W8_BYTES + 2 * nt * 128)
+    uint32_t ring_off;      // the BF16 weight ring, from the start of the stages
+};
+
+struct WoRange {
+    int32_t u0, cnt, nch;
+};
+
+__device__ __forceinline__ WoRange wo_range(int32_t units, int32_t c, int32_t ctas) {
+    const int32_t base = units / ctas, extra = units % ctas;
+    WoRange r;
+    r.u0 = c * base + min(c, extra);
+    r.cnt = base + (c < extra ? 1 : 0);
+    r.nch = (r.cnt + 7) / 8;
+    return r;
+}
+
+__device__ __forceinline__ void wo_chunk(const WoRange& r, int32_t j, int32_t& n0, int32_t& w) {
+    const int32_t ua = r.u0 + 8 * j;
+    const int32_t ub = min(ua + 8, r.u0 + r.cnt);
+    n0 = ua * WO_UNIT;
+    w = (ub - ua) * WO_UNIT;
+}
+
+// 16 FP8 codes (one 16-byte chunk) -> 16 BF16 values (two 16-byte chunks), exact.
+template <int WFMT>
+__device__ __forceinline__ void codes16_to_bf16(const uint4& c, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = decode_pair<WFMT>(w[i] & 0xFFFFu);
+        const float2 b = decode_pair<WFMT>(w[i] >> 16);
+        o[2 * i] = pack_bf16x2(a.x, a.y);
+        o[2 * i + 1] = pack_bf16x2(b.x, b.y);
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int WFMT>
+__global__ void __launch_bounds__(WO_THREADS, 1)
+fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW64,
+              const __grid_constant__ CUtensorMap tmW16, const GemmParams p, const WoParams d) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + WO_MAX_STAGES;
+    uint64_t* bfull = empty + WO_MAX_STAGES;
+    uint64_t* bempty = bfull + WO_SLOTS;
+    uint64_t* tfull = bempty + WO_SLOTS;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* teardown = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+    volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+    // stage s: FP8 W of WO_KBS K blocks (16 KB each), then X as 2 * WO_KBS BF16 halves
+    uint8_t* stages = smem + WO_BAR_BYTES;
+    uint8_t* ring = stages + d.ring_off;                 // WO_SLOTS x 16 KB of BF16 weight
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const WoRange range = wo_range(d.units, blockIdx.x, gridDim.x);
+    const int32_t S = d.stages;
+    const int32_t nkc = (p.num_kb + WO_KBS - 1) / WO_KBS;     // stages per chunk
+    const uint32_t x_off = WO_KBS * WO_W8_BYTES;
+    const uint32_t x_half = (uint32_t)d.nt * 128;               // bytes of one X half tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int t = 0; t < WO_SLOTS; ++t) {
+            ptx::mbar_init(&bfull[t], WO_CONV_WARPS);
+            ptx::mbar_init(&bempty[t], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], WO_EPI_WARPS);
+        }
+        ptx::mbar_init(teardown, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmX);
+        ptx::prefetch_tmap(&tmW64);
+        ptx::prefetch_tmap(&tmW16);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int32_t j = 0; j < range.nch && ok; ++j) {
+                int32_t n0, w;
+                wo_chunk(range, j, n0, w);
+                for (int32_t kc = 0; kc < nkc; ++kc) {
+                    const int32_t kb0 = kc * WO_KBS;
+                    const int32_t kbs = min(WO_KBS, p.num_kb - kb0);
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    uint8_t* st = stages + stage * d.stage_bytes;
+                    ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)kbs * ((uint32_t)w * BK + 2 * x_half));
+                    for (int32_t r = 0; r < w;) {
+                        const bool big = w - r >= 64;
+                        for (int32_t b = 0; b < kbs; ++b)
+                            ptx::tma_load_2d(st + b * WO_W8_BYTES + r * BK, big ? &tmW64 : &tmW16, &full[stage],
+                                             (kb0 + b) * BK, n0 + r);
+                        r += big ? 64 : WO_UNIT;
+                    }
+                    for (int32_t b = 0; b < kbs; ++b)
+                        for (int h = 0; h < 2; ++h)
+                            ptx::tma_load_2d(st + x_off + (2 * b + h) * x_half, &tmX, &full[stage],
+                                             (kb0 + b) * BK + h * 64, 0);
+                    if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer: D[n, m] += W_bf16 X^T
+        uint32_t stage = 0, phase = 0, acc_it = 0, conv_it = 0;
+        bool ok = true;
+        const uint32_t s0 = ptx::smem_u32(stages), r0 = ptx::smem_u32(ring);
+        for (int32_t j = 0; j < range.nch && ok; ++j) {
+            const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
+            if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            ptx::tc_fence_after();
+            for (int32_t kc = 0; kc < nkc && ok; ++kc) {
+                const int32_t kbs = min(WO_KBS, p.num_kb - kc * WO_KBS);
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                const uint32_t sx = s0 + stage * d.stage_bytes + x_off;
+                for (int32_t hb = 0; hb < 2 * kbs; ++hb) {
+                    const uint32_t t = conv_it % WO_SLOTS, tu = conv_it / WO_SLOTS;
+                    if (!wait_bounded(&bfull[t], tu & 1u, abort_flag, p.status)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {                       // K = 16 BF16 per instruction
+                            const uint64_t ad = ptx::sdesc_kmajor_sw128(r0 + t * WO_HALF_BYTES + k * 32);
+                            const uint64_t bd = ptx::sdesc_kmajor_sw128(sx + hb * x_half + k * 32);
+                            ptx::mma_f16(tmem_base + buf * 64, ad, bd, p.idesc, (kc | hb | k) != 0);
+                        }
+                        ptx::mma_commit(&bempty[t]);
+                    }
+                    __syncwarp();
+                    ++conv_it;
+                }
+                if (!ok) break;
+                if (lane == 0) ptx::mma_commit(&empty[stage]);
+                __syncwarp();
+                if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            if (lane == 0) ptx::mma_commit(&tfull[buf]);
+            __syncwarp();
+            ++acc_it;
+        }
+        if (lane == 0) {
+            ptx::mma_commit(teardown);
+            wait_bounded(teardown, 0, abort_flag, p.status);
+        }
+        __syncwarp();
+    } else if (warp < WO_FIRST_EPI) {
+        // ------------------------------------------------ converters: FP8 -> BF16 tiles
+        // thread ct owns row (ct % 128) and one half (ct / 128) of that row's 64 values
+        const int ct = threadIdx.x - 32 * WO_FIRST_CONV;
+        const int row = ct & 127, part = ct >> 7;
+        const int sw = row & 7;                              // the row's 128-byte swizzle phase
+        uint32_t stage = 0, phase = 0, conv_it = 0;
+        bool ok = true;
+        for (int32_t j = 0; j < range.nch && ok; ++j) {
+            for (int32_t kc = 0; kc < nkc && ok; ++kc) {
+                const int32_t kbs = min(WO_KBS, p.num_kb - kc * WO_KBS);
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                const uint8_t* w8 = stages + stage * d.stage_bytes;
+                for (int32_t hb = 0; hb < 2 * kbs; ++hb) {
+                    const uint32_t t = conv_it % WO_SLOTS, tu = conv_it / WO_SLOTS;
+                    if (!wait_bounded(&bempty[t], (tu & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    const int b = hb >> 1, h = hb & 1;
+                    const uint8_t* src = w8 + b * WO_W8_BYTES + row * 128;
+                    uint8_t* dst = ring + t * WO_HALF_BYTES + row * 128;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int jj = 2 * part + q;                 // 16-code chunk within this half
+                        const uint4 c = *reinterpret_cast<const uint4*>(src + (((4 * h + jj) ^ sw) * 16));
+                        uint4 lo, hi;
+                        codes16_to_bf16<WFMT>(c, lo, hi);
+                        *reinterpret_cast<uint4*>(dst + (((2 * jj) ^ sw) * 16)) = lo;
+                        *reinterpret_cast<uint4*>(dst + (((2 * jj + 1) ^ sw) * 16)) = hi;
+                    }
+                    ptx::fence_proxy_async_smem();               // generic writes -> tensor-core reads
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&bfull[t]);
+                    ++conv_it;
+                }
+                if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue: lane = weight row
+        const int quarter = warp & 3;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        uint32_t acc_it = 0;
+        for (int32_t j = 0; j < range.nch; ++j) {
+            int32_t n0, w;
+            wo_chunk(range, j, n0, w);
+            const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
+            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) break;
+            ptx::tc_fence_after();
+            const int32_t r = quarter * 32 + lane;
+            const int32_t n = n0 + r;
+            const bool valid = r < w && n < p.N;
+            if (quarter * 32 < w) {                                // warp-uniform
+                const float sw = valid ? __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
+                for (int32_t c0 = 0; c0 < p.M; c0 += 16) {
+                    uint32_t acc[16];
+                    ptx::tmem_ld_32x32b_x16(tmem_base + lane_base + buf * 64 + c0, acc);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int tk = 0; tk < 16; ++tk) {
+                        const int32_t m = c0 + tk;
+                        if (m < p.M && valid)
+                            p.y[(int64_t)m * p.ldy + n] = (uint16_t)(pack_bf16x2(__uint_as_float(acc[tk]) * sw, 0.0f) & 0xFFFFu);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+            ++acc_it;
+        }
+    }
+
+    // ------------------------------------------------ teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem_base, 128);
+}
+
+template <int WFMT>
+static cudaError_t launch_wo_t(const WoArgs& g, cudaStream_t st) {
+    GemmParams p{};
+    p.M = (int32_t)g.M;
+    p.N = (int32_t)g.N;
+    p.K = (int32_t)g.K;
+    p.num_kb = (int32_t)((g.K + BK - 1) / BK);
+    p.sb = static_cast<const float*>(g.sw);
+    p.sb_stride = g.w_row_scales ? 1 : 0;
+    p.status = g.status;
+    p.y = g.y;
+    p.ldy = g.ldy;
+    WoParams d{};
+    d.nt = (int32_t)((g.M + 15) / 16 * 16);
+    d.units = (int32_t)((g.N + WO_UNIT - 1) / WO_UNIT);
+    d.stage_bytes = WO_KBS * (WO_W8_BYTES + 2u * (uint32_t)d.nt * 128);
+    d.stages = (int32_t)std::min<uint32_t>(
+        WO_MAX_STAGES, (WO_SMEM - 1024 - WO_BAR_BYTES - WO_SLOTS * WO_HALF_BYTES) / d.stage_bytes);
+    d.ring_off = (uint32_t)d.stages * d.stage_bytes;
+    // BF16 x BF16 (kind::f16: formats 1 = BF16 in bits 7-9 and 10-12), FP32 D, M = 128, N = nt
+    p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(d.nt >> 3) << 17) | ((uint32_t)(WO_TILE >> 4) << 24);
+    CUtensorMap tx, t64, t16;
+    if (!make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.x, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.ldx * 2,
+                     64, (uint32_t)d.nt, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&t64, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&t16, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, 16,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(fp8_wo_kernel<WFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)WO_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    const uint32_t smem = 1024 + WO_BAR_BYTES + d.ring_off + WO_SLOTS * WO_HALF_BYTES;
+    const int grid = std::max(1, std::min(d.units, num_sms()));
+    fp8_wo_kernel<WFMT><<<grid, WO_THREADS, smem, st>>>(tx, t64, t16, p, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_weight_only(const WoArgs& g, cudaStream_t st) {
+    return g.w_fmt == FP8_E4M3 ? launch_wo_t<FP8_E4M3>(g, st) : launch_wo_t<FP8_E5M2>(g, st);
+}
+
+}  // namespace fp8b

@@ -275,6 +275,28 @@ FP8_API int32_t fp8_linear_forward_ex(const void* x_dev, int64_t M, int64_t K, i
                                       void* workspace_dev, size_t ws_bytes, void* stream);
 
 /*
+ * fp8_weight_only_linear -- weight-only FP8 linear for a few tokens:
+ *   y[m, n] = bf16( s_w[n] * sum_k x[m, k] * decode(w[n, k]) )
+ * with X in BF16 and only the weight in FP8 ([FFS] section "Weight-only FP8 与 W8A8
+ * FP8": the weight is stored in FP8, the activation stays BF16, the kernel reads
+ * the FP8 weight and converts it; the gain is the weight's memory and bandwidth).
+ * The weight codes are converted to BF16 on chip (exactly) and multiplied on the
+ * BF16 tensor-core path with FP32 accumulation; X is not quantised.
+ *   x_dev        bf16 [M, K], row stride ldx (ldx % 8 == 0), 16-byte aligned.
+ *   M            0 <= M <= FP8_WEIGHT_ONLY_MAX_TOKENS (the decode regime; larger
+ *                batches belong on fp8_linear_forward); K % 16 == 0.
+ *   w_dev, w_scale_dev, w_mode, w_fmt: codes [N, K] and the TENSOR / ROW (or
+ *                DELAYED, read as TENSOR) scale fp8_quantize produced; E4M3 or E5M2.
+ *   y_dev        bf16 [M, N], row stride ldy >= N.  K == 0 writes zeros.
+ *   dev_status   nullable; FP8_ERR_TIMEOUT if a pipeline wait gave up.
+ * No workspace.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ */
+#define FP8_WEIGHT_ONLY_MAX_TOKENS 64
+FP8_API int32_t fp8_weight_only_linear(const void* x_dev, int64_t M, int64_t K, int64_t ldx, const uint8_t* w_dev,
+                                       const void* w_scale_dev, int32_t w_mode, int32_t w_fmt, int64_t N,
+                                       void* y_dev, int64_t ldy, int32_t* dev_status, void* stream);
+
+/*
  * fp8_linear_forward_noalloc -- fp8_linear_forward for callers that cannot
  * allocate device memory.  (The source pages have no counterpart: this is a
  * deployment convenience of this library, not part of the method.)
