@@ -43,6 +43,7 @@ struct GemmParams {
     int64_t ldy;
     int32_t y_direct;
     int32_t y_vec;          // y rows start 16-byte aligned (ldy % 8 == 0, aligned base)
+    int32_t sb_vec;         // per-row b scales start 16-byte aligned
     // optional epilogue (fp8_epilogue_t); ext != 0 when any option is set
     int32_t ext;
     int32_t write_y;        // 0: no bf16 Y (FP8 output only)
@@ -53,7 +54,8 @@ struct GemmParams {
     int64_t ldq;
     int32_t yq_fmt;
     int32_t yq_vec;         // yq rows start 16-byte aligned
-    // launched as the programmatic dependent of the kernel that produced A (and only A)
+    // launched as the programmatic dependent of the kernel that produced A (and only A);
+    // every kernel waits (pdl_wait) before it reads A or the scales
     int32_t pdl;
 };
 
@@ -229,6 +231,24 @@ template <bool EXT>
 __device__ __forceinline__ void rowscale_chunk(const GemmParams& p, EpiState& es, const uint32_t (&r)[32], float sx,
                                                int32_t n0, int32_t n_lim, int32_t row, uint32_t (&w)[16]) {
     if constexpr (!EXT) {
+        if (n0 + 32 <= n_lim && (p.sb_stride == 0 || p.sb_vec)) {
+            // whole chunk: the 32 channel scales as eight 16-byte loads (the same for
+            // every lane), products on f32x2 pairs; the same roundings as below
+            const float2 sx2 = make_float2(sx, sx);
+            const float4* sb4 = reinterpret_cast<const float4*>(p.sb + n0);
+            const float sb0 = p.sb_stride == 0 ? __ldg(p.sb) : 0.0f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 b = p.sb_stride == 0 ? make_float4(sb0, sb0, sb0, sb0) : __ldg(sb4 + q);
+                const float2 s01 = mul2_rn(sx2, make_float2(b.x, b.y));
+                const float2 s23 = mul2_rn(sx2, make_float2(b.z, b.w));
+                const float2 v01 = mul2_rn(make_float2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), s01);
+                const float2 v23 = mul2_rn(make_float2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), s23);
+                w[2 * q] = pack_bf16x2(v01.x, v01.y);
+                w[2 * q + 1] = pack_bf16x2(v23.x, v23.y);
+            }
+            return;
+        }
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
             const int32_t n = n0 + j;

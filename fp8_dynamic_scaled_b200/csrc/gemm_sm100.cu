@@ -144,6 +144,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            pdl_wait();                       // A may come from the kernel just before
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -223,6 +224,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         __syncwarp();
     } else if (V == V_MX && warp == 2) {
         // ------------------------------------------------ MX scale-factor warp
+        pdl_wait();
         // Stage layout (what tcgen05.cp 32x128b.warpx4 reads): for a block of 128
         // rows, byte (r % 32) * 16 + (r / 32) * 4 + j holds the scale of row r for
         // the j-th 32-wide K slice of this 128-wide stage.
@@ -314,6 +316,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     } else {
         // ------------------------------------------------ epilogue
         if (V == V_BLOCK) ptx::regs_inc<224>();
+        pdl_wait();                           // the scales may come from the kernel just before
         const int ew = warp - C::FIRST_EPI_WARP;          // 0 .. EPI_WARPS-1
         const int quarter = warp & 3;                      // TMEM lane quarter this warp may access
         const int half = (C::EPI_WARPS == 8) ? (ew >> 2) : 0;   // column half (8-warp variants)
@@ -577,6 +580,7 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
+            pdl_wait();                       // A may come from the kernel just before
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
@@ -642,6 +646,7 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
     } else {
         // ------------------------------------------------ epilogue (both CTAs)
+        pdl_wait();                           // the scales may come from the kernel just before
         const int ew = warp - S::FIRST_EPI_WARP;
         const int quarter = warp & 3;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -717,7 +722,18 @@ static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaSt
     }
     const int32_t tiles = p.num_m * p.num_n;
     const int grid = std::max(1, std::min(tiles, num_sms()));
-    fp8_gemm_kernel<V, EXT><<<grid, Smem<V>::NT, Smem<V>::ALLOC, st>>>(ta, tb, ty, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(Smem<V>::NT);
+    cfg.dynamicSmemBytes = Smem<V>::ALLOC;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;      // dependent of the quantize kernel that wrote A
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<V, EXT>, ta, tb, ty, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -774,13 +790,15 @@ static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st)
     cfg.blockDim = dim3(PairSmem::NT);
     cfg.dynamicSmemBytes = PairSmem::ALLOC;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = p.pdl ? 2 : 1;      // dependent of the quantize kernel that wrote A
     cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_pair_kernel<EXT>, ta, tb, ty, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -829,6 +847,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
     p.status = g.status;
     p.y = g.y;
     p.ldy = g.ldy;
+    p.pdl = g.a_from_previous_kernel ? 1 : 0;
     p.y_vec = (g.ldy % 8 == 0 && (reinterpret_cast<uintptr_t>(g.y) & 15u) == 0) ? 1 : 0;
     p.y_direct = p.y_vec ? 0 : 1;
     set_epilogue(g, p);
@@ -839,13 +858,11 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
         p.sb = static_cast<const float*>(g.sb);
         p.sa_stride = a_pt ? 0 : 1;
         p.sb_stride = b_pt ? 0 : 1;
+        p.sb_vec = (reinterpret_cast<uintptr_t>(g.sb) & 15u) == 0 ? 1 : 0;
         p.idesc = idesc_f8f6f4(g.fmt_a, g.fmt_b);
         // a few tokens: stream W across all SMs; CTA pairs once M spans a 256-row tile;
         // a single CTA per tile in between
-        if (g.M <= D_MAX_TOKENS) {
-            p.pdl = g.a_from_previous_kernel ? 1 : 0;
-            return launch_decode(g, p, st);
-        }
+        if (g.M <= D_MAX_TOKENS) return launch_decode(g, p, st);
         if (g.M >= P_BM) return p.ext ? launch_pair<true>(g, p, st) : launch_pair<false>(g, p, st);
         return p.ext ? launch_variant<V_ROWSCALE, true>(g, p, st) : launch_variant<V_ROWSCALE, false>(g, p, st);
     }

@@ -692,7 +692,7 @@ __global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(
         } else {
             cq = cast_vec_rcp<FMT>(a, op);
         }
-        *reinterpret_cast<uint2*>(p.q + vv * VEC) = cq;
+        __stcs(reinterpret_cast<uint2*>(p.q + vv * VEC), cq);   // evict-first: keep X in L2 for the pass
         if (DEQ) st_v4_stream(p.deq + vv * VEC, dequant_vec2<FMT>(cq, s));
     };
     int64_t t = (int64_t)blockIdx.x * QT + threadIdx.x;
@@ -724,6 +724,48 @@ __global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(
                 *reinterpret_cast<volatile uint32_t*>(p.pending) = 0u;
                 *reinterpret_cast<volatile uint32_t*>(p.ticket) = 0u;
             }
+        }
+    }
+}
+
+// Per-tensor current scaling of a small dense tensor (<= 1024 * SMALL_VPT vectors) in
+// one CTA: the whole tensor stays in registers through the block-wide amax and the
+// cast, so the two launches of the large-tensor path become one.  Same arithmetic
+// as rq_amax_kernel + rq_tensor_kernel<RQ_CAST> (codes and scale bit for bit).
+constexpr int SMALL_VPT = 8;
+constexpr int SMALL_THREADS = 1024;
+
+template <int FMT, bool DEQ>
+__global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const RQParams p) {
+    pdl_launch_dependents();   // a dependent GEMM may start streaming its other operand
+    __shared__ uint32_t red[32];
+    const int64_t nvec = p.n / VEC;
+    uint4 v[SMALL_VPT];
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int j = 0; j < SMALL_VPT; ++j) {
+        const int64_t k = threadIdx.x + (int64_t)SMALL_THREADS * j;
+        v[j] = k < nvec ? ld_v4(p.x + k * VEC) : make_uint4(0, 0, 0, 0);
+        m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(v[j]));
+    }
+    uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
+    if (m >= 0x7F80u) {
+        if (threadIdx.x == 0) report_status(p.status, FP8_ERR_NONFINITE);
+        m = 0x7F7Fu;
+    }
+    const float amax = bf16bits_to_float(m);
+    const RcpScale op = rcp_scale_from_amax_bits<FMT>(m);
+    if (threadIdx.x == 0) {
+        reinterpret_cast<float*>(p.scale)[0] = op.s;
+        if (p.ring != nullptr) p.ring[p.slot] = amax;          // delayed scaling, step 0
+    }
+#pragma unroll
+    for (int j = 0; j < SMALL_VPT; ++j) {
+        const int64_t k = threadIdx.x + (int64_t)SMALL_THREADS * j;
+        if (k < nvec) {
+            const uint2 cq = cast_vec_rcp<FMT>(v[j], op);
+            *reinterpret_cast<uint2*>(p.q + k * VEC) = cq;
+            if (DEQ) st_v4_stream(p.deq + k * VEC, dequant_vec2<FMT>(cq, op.s));
         }
     }
 }
@@ -790,6 +832,10 @@ static cudaError_t rq_tensor_t(const QuantArgs& a, cudaStream_t st) {
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rq_grid_cap(), (nvec + QT - 1) / QT));
     if (a.hist_ring != nullptr && a.hist_step > 0) {
         rq_tensor_kernel<FMT, DEQ, RQ_DELAYED, 4><<<(unsigned)grid, QT, 0, st>>>(p);
+        return cudaGetLastError();
+    }
+    if (nvec <= (int64_t)SMALL_THREADS * SMALL_VPT) {
+        rq_small_tensor_kernel<FMT, DEQ><<<1, SMALL_THREADS, 0, st>>>(p);
         return cudaGetLastError();
     }
     rq_amax_kernel<8><<<(unsigned)grid, QT, 0, st>>>(p);
