@@ -208,6 +208,20 @@ def test_delayed_sixteen_steps_small(fmt):
     run_delayed_sequence(xs, fmt)
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(256, 256), (64, 1024), (32, 2048 + 16), (1, 8192 * 8), (2, 8192 * 4 + 16)])
+def test_per_tensor_around_the_single_cta_limit(fmt, shape):
+    """Dense per-tensor tensors up to 65,536 elements take the one-CTA kernel, larger ones
+    the two-pass kernels; both sides of the limit against the oracle."""
+    check_parity(mixed_input(*shape, seed=sum(shape)), fmt, fp8.FP8_SCALE_TENSOR, what=f"per-tensor {shape}")
+
+
+def test_delayed_small_tensor_single_cta():
+    """Step 0 of a small delayed tensor runs in the one-CTA kernel and must record amax_0."""
+    xs = [inputs.delayed_step_input(t, M=64, K=256) for t in range(6)]
+    run_delayed_sequence(xs, fp8.FP8_E5M2, hist_len=4)
+
+
 def test_delayed_short_history_and_strided_grid():
     xs = [mixed_input(1000, 1024, seed=t) for t in range(7)]
     run_delayed_sequence(xs, fp8.FP8_E4M3, hist_len=3)
