@@ -134,6 +134,15 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 // dependent) has completed and its writes are visible; a no-op otherwise.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Host: the current device as an index into small per-device caches (kernel
+// attributes, SM counts), or -1 when it is outside them (then nothing is cached).
+constexpr int kDeviceCacheSlots = 64;
+inline int device_slot() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kDeviceCacheSlots) return -1;
+    return d;
+}
+
 // Record the first device-side error in a caller-owned status word.
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
     if (status) atomicCAS(status, 0, code);

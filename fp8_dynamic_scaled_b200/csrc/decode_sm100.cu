@@ -285,12 +285,13 @@ static cudaError_t launch_decode_t(const GemmArgs& g, GemmParams p, cudaStream_t
         !make_map_2d(&t16, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, 16,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    static bool attr_done = false;
-    if (!attr_done) {
+    static bool attr_done[kDeviceCacheSlots];   // the attribute is set per device
+    const int ds = device_slot();
+    if (ds < 0 || !attr_done[ds]) {
         cudaError_t e = cudaFuncSetAttribute(fp8_decode_kernel<EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)D_SMEM);
         if (e != cudaSuccess) return e;
-        attr_done = true;
+        if (ds >= 0) attr_done[ds] = true;
     }
     // request only what the stages use, so that a small kernel running just before (the
     // X quantize, whose dependent this kernel may be) can share an SM with this one

@@ -259,10 +259,28 @@ __device__ __forceinline__ void rowscale_chunk(const GemmParams& p, EpiState& es
     } else {
         // columns at or past n_lim are zero (their accumulators may hold anything)
         float f[32];
+        if (n0 + 32 <= n_lim && (p.sb_stride == 0 || p.sb_vec)) {
+            const float2 sx2 = make_float2(sx, sx);
+            const float4* sb4 = reinterpret_cast<const float4*>(p.sb + n0);
+            const float sb0 = p.sb_stride == 0 ? __ldg(p.sb) : 0.0f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int32_t n = n0 + j;
-            f[j] = n < n_lim ? __uint_as_float(r[j]) * (sx * __ldg(p.sb + (int64_t)n * p.sb_stride)) : 0.0f;
+            for (int q = 0; q < 8; ++q) {
+                const float4 b = p.sb_stride == 0 ? make_float4(sb0, sb0, sb0, sb0) : __ldg(sb4 + q);
+                const float2 v01 = mul2_rn(make_float2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])),
+                                           mul2_rn(sx2, make_float2(b.x, b.y)));
+                const float2 v23 = mul2_rn(make_float2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])),
+                                           mul2_rn(sx2, make_float2(b.z, b.w)));
+                f[4 * q] = v01.x;
+                f[4 * q + 1] = v01.y;
+                f[4 * q + 2] = v23.x;
+                f[4 * q + 3] = v23.y;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int32_t n = n0 + j;
+                f[j] = n < n_lim ? __uint_as_float(r[j]) * (sx * __ldg(p.sb + (int64_t)n * p.sb_stride)) : 0.0f;
+            }
         }
         epi_chunk(p, es, f, n0, n_lim, row, w);
     }
@@ -300,13 +318,14 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
 }
 
 static int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    static int cache[kDeviceCacheSlots];
+    const int ds = device_slot();
+    if (ds >= 0 && cache[ds] > 0) return cache[ds];
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    if (ds >= 0) cache[ds] = n;
     return n;
 }
 

@@ -713,12 +713,13 @@ static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaSt
     if (!p.y_direct && !make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, (uint64_t)g.N, (uint64_t)g.M,
                                     (uint64_t)g.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
-    static bool attr_done = false;
-    if (!attr_done) {
+    static bool attr_done[kDeviceCacheSlots];   // the attribute is set per device
+    const int ds = device_slot();
+    if (ds < 0 || !attr_done[ds]) {
         cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<V, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)Smem<V>::ALLOC);
         if (e != cudaSuccess) return e;
-        attr_done = true;
+        if (ds >= 0) attr_done[ds] = true;
     }
     const int32_t tiles = p.num_m * p.num_n;
     const int grid = std::max(1, std::min(tiles, num_sms()));
@@ -762,7 +763,9 @@ static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st)
     if (!p.y_direct && !make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, (uint64_t)g.N, (uint64_t)g.M,
                                     (uint64_t)g.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
-    static int max_clusters = 0;
+    static int max_clusters_of[kDeviceCacheSlots];   // per device
+    const int ds = device_slot();
+    int max_clusters = ds >= 0 ? max_clusters_of[ds] : 0;
     if (max_clusters == 0) {
         cudaError_t e = cudaFuncSetAttribute(fp8_gemm_pair_kernel<EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)PairSmem::ALLOC);
@@ -782,6 +785,7 @@ static cudaError_t launch_pair(const GemmArgs& g, GemmParams p, cudaStream_t st)
         e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_pair_kernel<EXT>, &q);
         if (e != cudaSuccess || n <= 0) n = num_sms() / 2;
         max_clusters = n;
+        if (ds >= 0) max_clusters_of[ds] = n;
     }
     const int32_t tiles = p.num_m * p.num_n;
     const int clusters = std::max(1, std::min(tiles, max_clusters));

@@ -772,13 +772,14 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const
 
 // ================================================================ launchers
 static int sm_count_cached() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    static int cache[kDeviceCacheSlots];   // per device
+    const int ds = device_slot();
+    if (ds >= 0 && cache[ds] > 0) return cache[ds];
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    if (ds >= 0) cache[ds] = n;
     return n;
 }
 

@@ -317,12 +317,13 @@ static cudaError_t launch_wo_t(const WoArgs& g, cudaStream_t st) {
         !make_map_2d(&t16, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K, (uint64_t)g.N, (uint64_t)g.K, BK, 16,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    static bool attr_done = false;
-    if (!attr_done) {
+    static bool attr_done[kDeviceCacheSlots];   // the attribute is set per device
+    const int ds = device_slot();
+    if (ds < 0 || !attr_done[ds]) {
         cudaError_t e = cudaFuncSetAttribute(fp8_wo_kernel<WFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)WO_SMEM);
         if (e != cudaSuccess) return e;
-        attr_done = true;
+        if (ds >= 0) attr_done[ds] = true;
     }
     const uint32_t smem = 1024 + WO_BAR_BYTES + d.ring_off + WO_SLOTS * WO_HALF_BYTES;
     const int grid = std::max(1, std::min(d.units, num_sms()));
