@@ -5,13 +5,15 @@ the quantisation or GEMM arithmetic.  Both the CUDA path (through the tests and
 the benchmark) and the CPU oracle take their inputs from here, so the two
 always see the same bits.
 
-Workloads (sizes and distributions as the design notes state them):
+Workloads (sizes and value distributions):
   * ``linear_small``      X [128, 256] ~ N(0,1) with one element set to 400.0,
                           W [256, 256] ~ N(0, 0.02).
   * ``quant_sweep``       64 Mi elements ([8192, 8192]) with |x| = 10^U(-6, 4),
                           random signs, round(1e-4 * n) outliers at +-1e5.
   * ``llama70b_prefill``  X [4096, 8192] ~ N(0,1) with 0.1% of the channels (8)
-                          scaled x50, W [28672, 8192] ~ N(0, 0.02).
+                          scaled x50, W [28672, 8192] ~ N(0, 0.02).  The decode
+                          shape is the same recipe with M = 16 (1 to 64 tokens in
+                          the decode tests).
   * ``block_scaled``      X [8192, 8192] and W [28672, 8192]; value = N(0,1) times
                           one lognormal(0,1) draw per scaling block (1x128 for X,
                           128x128 for W).

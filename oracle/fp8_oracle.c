@@ -23,7 +23,7 @@
  *         section "数值特性" (bias 7 / 15; E5M2 full Inf/NaN, E4M3 limited);
  *         section "量化流程" (x / s, round to an FP8 value, store).
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings where the pages are silent:
  *  - rounding is IEEE round-to-nearest, ties to even mantissa;
  *  - E4M3 is the "fn" variant: no Inf, NaN only at S.1111.111, subnormals kept;
  *  - E5M2 follows IEEE-754 binary conventions (Inf at S.11111.00, NaN above);
@@ -34,8 +34,9 @@
  *  - delayed: step 0 uses the current amax, later steps the max over the ring,
  *    and amax_t of the raw input is written to ring[t mod h] after use.
  *
- * Parity status: every function here is pinned by tests under tests/ (see the
- * pin list in the design notes); none is "parity unpinned".
+ * Parity status: every function here is pinned (tests/test_oracle_pins.py and
+ * tests/test_oracle_epilogue_pins.py: printed examples under tests/golden, closed
+ * forms, exact integer arithmetic, brute force); none is "parity unpinned".
  */
 #include <math.h>
 #include <stdint.h>
