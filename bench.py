@@ -511,8 +511,9 @@ def extras(torch, fp8, stream, peaks):
                     torch.cuda.synchronize()
                     per[k].append(a.elapsed_time(b) / 50 * 1e3)
             res[f"layer_M{Md}_us"] = {k: statistics.median(v) for k, v in per.items()}
-        # weight-only FP8 (X stays bf16, W codes converted on chip): the same layer
-        for Md in (1, 16, 64):
+        # weight-only FP8 (X stays bf16, W codes decoded on chip): the same layer; up to
+        # 3 tokens on the CUDA-core matrix-vector kernel, above on the tensor-core one
+        for Md in (1, 2, 3, 4, 16, 64):
             xd = to_dev_bf16(torch, xh_all[:Md])
             yd = torch.empty((Md, N), dtype=torch.bfloat16, device="cuda")
             med, _ = time_kernel(torch, lambda: fp8.fp8_weight_only_linear(xd, wq, wsc, fp8.FP8_SCALE_ROW, fp8.FP8_E4M3,

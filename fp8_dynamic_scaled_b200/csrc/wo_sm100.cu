@@ -20,6 +20,12 @@
 //   - the epilogue warp of a TMEM lane quarter owns 32 weight rows and writes
 //     bf16(acc * s_w[n]) for every token.
 // Every wait is bounded as in the other kernels.
+//
+// Up to WG_MAX_TOKENS (3) tokens the product is a matrix-vector one whose bound is
+// the weight's bytes, and a tcgen05.mma with N = 16 (the smallest at M = 128) moves only
+// 2 KB of FP8 weight per instruction as BF16; there fp8_wo_gemv_kernel does the
+// contraction on the CUDA cores instead: W streamed once with 16-byte loads, codes
+// decoded in registers, FP32 accumulation on packed f32x2 FMAs.
 #include "gemm_common.cuh"
 
 namespace fp8b {
@@ -331,7 +337,137 @@ static cudaError_t launch_wo_t(const WoArgs& g, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// ================================================================ matrix-vector path
+// A warp owns 8 consecutive weight rows.  Lane l works on rows (l >> 3) and
+// (l >> 3) + 4 of them and on the 16-code chunk (l & 7) of every 128-code step, so
+// the 8 lanes of a row read one full 128-byte line of it per step and each lane
+// converts its X chunk once for two rows.  After the K loop the 8 partial sums of
+// a row are added with shuffles and lane (l & 7) == 0 writes bf16(sum * s_w[n]).
+// Loads are in bounds by construction: n < N, k0 + 16 <= K (K % 16 == 0), m < M.
+constexpr int WG_THREADS = 256;
+constexpr int WG_MAX_TOKENS = 3;                        // measured: at 4 tokens the tensor-core kernel ties
+
+template <int MT>
+struct WgShape {
+    static constexpr int U = MT <= 2 ? 2 : 1;           // 128-code steps in flight per lane (measured)
+};
+
+template <int WFMT, int MT>
+__global__ void __launch_bounds__(WG_THREADS, 4)
+fp8_wo_gemv_kernel(const uint16_t* __restrict__ x, int64_t ldx, const uint8_t* __restrict__ w,
+                   const float* __restrict__ sw, int32_t sw_stride, int32_t N, int32_t K,
+                   uint16_t* __restrict__ y, int64_t ldy) {
+    constexpr int U = WgShape<MT>::U;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane & 7, slot = lane >> 3;
+    const int64_t warp0 = ((int64_t)blockIdx.x * WG_THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * WG_THREADS) >> 5;
+    const int64_t groups = ((int64_t)N + 7) / 8;
+    const int32_t steps = (K + 127) / 128;
+    for (int64_t g = warp0; g < groups; g += nwarps) {            // warp-uniform
+        const int32_t n0 = (int32_t)(g * 8) + slot, n1 = n0 + 4;
+        const bool v0 = n0 < N, v1 = n1 < N;
+        const uint8_t* w0 = w + (int64_t)(v0 ? n0 : 0) * K;
+        const uint8_t* w1 = w + (int64_t)(v1 ? n1 : 0) * K;
+        float2 acc[MT][2];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[m][0] = acc[m][1] = make_float2(0.0f, 0.0f);
+        for (int32_t s = 0; s < steps; s += U) {
+            uint4 a[U][2];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t k0 = (int64_t)(s + u) * 128 + sub * 16;
+                const bool kin = k0 < K;
+                a[u][0] = (kin && v0) ? __ldcs(reinterpret_cast<const uint4*>(w0 + k0)) : make_uint4(0, 0, 0, 0);
+                a[u][1] = (kin && v1) ? __ldcs(reinterpret_cast<const uint4*>(w1 + k0)) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t k0 = (int64_t)(s + u) * 128 + sub * 16;
+                if (k0 >= K) continue;
+                // the chunk in two halves of 8 codes, so that few decoded values are live
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // codes 8h + 2q and 8h + 2q + 1 -> wf[r][q]
+                    float2 wf[2][4];
+                    const uint32_t c0[2] = {h ? a[u][0].z : a[u][0].x, h ? a[u][0].w : a[u][0].y};
+                    const uint32_t c1[2] = {h ? a[u][1].z : a[u][1].x, h ? a[u][1].w : a[u][1].y};
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        wf[0][2 * i] = decode_pair<WFMT>(c0[i] & 0xFFFFu);
+                        wf[0][2 * i + 1] = decode_pair<WFMT>(c0[i] >> 16);
+                        wf[1][2 * i] = decode_pair<WFMT>(c1[i] & 0xFFFFu);
+                        wf[1][2 * i + 1] = decode_pair<WFMT>(c1[i] >> 16);
+                    }
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        const uint4 xv4 = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)m * ldx + k0 + 8 * h));
+                        const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            // bf16 pair -> exact fp32 pair (the even value in the low half)
+                            const float2 xf =
+                                make_float2(__uint_as_float(xv[q] << 16), __uint_as_float(xv[q] & 0xFFFF0000u));
+                            acc[m][0] = ptx::ffma2(xf, wf[0][q], acc[m][0]);
+                            acc[m][1] = ptx::ffma2(xf, wf[1][q], acc[m][1]);
+                        }
+                    }
+                }
+            }
+        }
+        const float s0 = v0 ? __ldg(sw + (int64_t)n0 * sw_stride) : 0.0f;
+        const float s1 = v1 ? __ldg(sw + (int64_t)n1 * sw_stride) : 0.0f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float t0 = acc[m][0].x + acc[m][0].y, t1 = acc[m][1].x + acc[m][1].y;
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                t0 += __shfl_xor_sync(0xFFFFFFFFu, t0, o);
+                t1 += __shfl_xor_sync(0xFFFFFFFFu, t1, o);
+            }
+            if (sub == 0) {
+                if (v0) y[(int64_t)m * ldy + n0] = (uint16_t)(pack_bf16x2(t0 * s0, 0.0f) & 0xFFFFu);
+                if (v1) y[(int64_t)m * ldy + n1] = (uint16_t)(pack_bf16x2(t1 * s1, 0.0f) & 0xFFFFu);
+            }
+        }
+    }
+}
+
+template <int WFMT, int MT>
+static cudaError_t launch_gemv_t(const WoArgs& g, cudaStream_t st) {
+    static int per_sm_of[kDeviceCacheSlots];              // resident CTAs per SM, per device
+    const int ds = device_slot();
+    int per_sm = ds >= 0 ? per_sm_of[ds] : 0;
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8_wo_gemv_kernel<WFMT, MT>, WG_THREADS, 0) !=
+                cudaSuccess ||
+            per_sm <= 0)
+            per_sm = 1;
+        if (ds >= 0) per_sm_of[ds] = per_sm;
+    }
+    const int64_t groups = (g.N + 7) / 8;
+    const int64_t want = (groups + WG_THREADS / 32 - 1) / (WG_THREADS / 32);      // one row group per warp
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)num_sms() * per_sm));
+    fp8_wo_gemv_kernel<WFMT, MT><<<grid, WG_THREADS, 0, st>>>(g.x, g.ldx, g.w, static_cast<const float*>(g.sw),
+                                                              g.w_row_scales ? 1 : 0, (int32_t)g.N, (int32_t)g.K,
+                                                              g.y, g.ldy);
+    return cudaGetLastError();
+}
+
+template <int WFMT>
+static cudaError_t launch_gemv(const WoArgs& g, cudaStream_t st) {
+    static_assert(WG_MAX_TOKENS == 3, "one instantiation per token count");
+    switch (g.M) {
+        case 1: return launch_gemv_t<WFMT, 1>(g, st);
+        case 2: return launch_gemv_t<WFMT, 2>(g, st);
+        case 3: return launch_gemv_t<WFMT, 3>(g, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_weight_only(const WoArgs& g, cudaStream_t st) {
+    if (g.M <= WG_MAX_TOKENS)
+        return g.w_fmt == FP8_E4M3 ? launch_gemv<FP8_E4M3>(g, st) : launch_gemv<FP8_E5M2>(g, st);
     return g.w_fmt == FP8_E4M3 ? launch_wo_t<FP8_E4M3>(g, st) : launch_wo_t<FP8_E5M2>(g, st);
 }
 

@@ -280,8 +280,10 @@ FP8_API int32_t fp8_linear_forward_ex(const void* x_dev, int64_t M, int64_t K, i
  * with X in BF16 and only the weight in FP8 ([FFS] section "Weight-only FP8 与 W8A8
  * FP8": the weight is stored in FP8, the activation stays BF16, the kernel reads
  * the FP8 weight and converts it; the gain is the weight's memory and bandwidth).
- * The weight codes are converted to BF16 on chip (exactly) and multiplied on the
- * BF16 tensor-core path with FP32 accumulation; X is not quantised.
+ * X is not quantised; the weight codes are decoded on chip (exactly) and the
+ * products are accumulated in FP32.  Up to 3 tokens the contraction runs on the
+ * CUDA cores (a matrix-vector product bound by the weight's bytes); above that the
+ * codes are converted to BF16 and multiplied on the BF16 tensor-core path.
  *   x_dev        bf16 [M, K], row stride ldx (ldx % 8 == 0), 16-byte aligned.
  *   M            0 <= M <= FP8_WEIGHT_ONLY_MAX_TOKENS (the decode regime; larger
  *                batches belong on fp8_linear_forward); K % 16 == 0.

@@ -4,9 +4,12 @@ X stays BF16; the weight is FP8 codes with a per-tensor or per-row scale (quanti
 by the oracle here, so the test does not lean on the GPU quantiser).  Reference: the
 oracle's fp64 sum of x times the decoded, scaled weight, under the usual acceptance
 rule |y - y_ref| <= 1e-3 * sum_k |terms| + 1 bf16 ulp; exact integer cases are
-compared bit for bit.  The shapes hit one-unit and uneven per-SM ranges, several
-chunks per CTA, ragged N and K (a last stage with fewer K blocks, a half-empty
-last K block) and token counts up to the maximum."""
+compared bit for bit.  Up to 3 tokens the CUDA-core matrix-vector kernel runs,
+above that the tensor-core one; the token counts cover both sides of the switch.
+The shapes hit one-unit and uneven per-SM ranges, several chunks per CTA, ragged N
+(not a multiple of the 8-row groups) and K (a last stage with fewer K blocks, a
+half-empty last K block, K below one 128-code step) and token counts up to the
+maximum."""
 import numpy as np
 import pytest
 import torch
@@ -64,28 +67,31 @@ def check(M, N, K, mode, fmt, seed, ldx=None, ldy=None):
     assert_gemm_close(y, y_ref, bound, f"weight-only {M}x{N}x{K} mode {mode} fmt {fmt}")
 
 
-@pytest.mark.parametrize("M", [1, 2, 16, 33, 64])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 16, 33, 64])
 @pytest.mark.parametrize("N,K", [(16, 128), (200, 512), (2368, 256), (3000, 640), (1000, 1040), (300, 16),
-                                 (20000, 1152)])
+                                 (20000, 1152), (13, 48), (4099, 400)])
 def test_weight_only_shapes(M, N, K):
     check(M, N, K, R, E4M3, seed=M * 13 + N + K)
 
 
+@pytest.mark.parametrize("M", [4, 16])
 @pytest.mark.parametrize("mode", [T, R])
 @pytest.mark.parametrize("fmt", [E4M3, E5M2])
-def test_weight_only_modes_and_formats(mode, fmt):
-    check(16, 1500, 768, mode, fmt, seed=7 + fmt)
+def test_weight_only_modes_and_formats(M, mode, fmt):
+    check(M, 1500, 768, mode, fmt, seed=7 + fmt + M)
 
 
-def test_weight_only_strides():
-    check(9, 700, 512, R, E4M3, seed=3, ldx=512 + 24, ldy=700 + 40)
-    check(9, 700, 512, R, E4M3, seed=4, ldy=703)
+@pytest.mark.parametrize("M", [3, 9])
+def test_weight_only_strides(M):
+    check(M, 700, 512, R, E4M3, seed=3, ldx=512 + 24, ldy=700 + 40)
+    check(M, 700, 512, R, E4M3, seed=4, ldy=703)
 
 
-def test_weight_only_exact_integer():
+@pytest.mark.parametrize("M", [1, 6, 16])
+def test_weight_only_exact_integer(M):
     """Integer activations (exact in bf16) and integer codes with unit scale: exact."""
-    g = np.random.default_rng(61)
-    M, N, K = 16, 512, 256
+    g = np.random.default_rng(61 + M)
+    N, K = 512, 256
     x_int = g.integers(-2, 3, (M, K)).astype(np.float32)
     w_int = g.integers(-2, 3, (N, K)).astype(np.float32)
     x = inputs.bf16_bits(x_int)
@@ -118,7 +124,7 @@ def test_weight_only_empty_zero_k_and_bad_args():
     assert e.value.status == fp8.FP8_ERR_ALIGNMENT
 
 
-@pytest.mark.parametrize("M", [1, 16, 64])
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 64])
 def test_weight_only_llama70b_layer_full_size(M):
     """M tokens against the whole 28672 x 8192 weight (per-channel scales), every output
     of 2,048 sampled weight rows against the oracle."""
