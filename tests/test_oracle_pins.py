@@ -133,6 +133,38 @@ def test_fpi_dequant_worked_example(fmt, col):
     assert np.all(np.abs(deq.astype(np.float64) - printed) <= ulp)
 
 
+@pytest.mark.parametrize("fmt,col", [(E4M3, 2), (E5M2, 3)])
+def test_dequant_scaled_worked_example(fmt, col):
+    """[FPI] "反量化示例" through the oracle's dequantiser: bf16 of fp32(decode(q) * 0.01)
+    lies within one bf16 step of the printed 0.0125, -0.005, 0.03."""
+    rows, table = read_golden("fpi_dequant_example.txt")
+    codes = np.array([int(r[col], 16) for r in table], np.uint8)
+    printed = np.array([float(r[1]) for r in table])
+    got = oracle.bf16_to_f32(oracle.dequant_scaled(codes, float(rows["scale"][0]), fmt)).astype(np.float64)
+    step = np.array([oracle.bf16_ulp(v) for v in printed])
+    assert np.all(np.abs(got - printed) <= step)
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_dequant_scaled_exact_cases_and_torch(fmt):
+    """Every FP8 value is a bf16 value, so a unit or power-of-two scale dequantises
+    exactly; NaN codes stay NaN and E5M2's infinities stay infinite; any other scale
+    gives the bf16 rounding of the fp32 product, as torch computes it."""
+    codes = np.arange(256, dtype=np.uint8)
+    table = oracle.decode_table(fmt)
+    fin = np.isfinite(table)
+    for k in (0, -7, 5, -20):
+        got = oracle.bf16_to_f32(oracle.dequant_scaled(codes, 2.0 ** k, fmt)).astype(np.float64)
+        assert np.array_equal(got[fin], table[fin] * 2.0 ** k)
+        assert np.all(np.isnan(got[np.isnan(table)]))
+        assert np.array_equal(got[np.isinf(table)], table[np.isinf(table)])
+    g = np.random.default_rng(71 + fmt)
+    for s in np.float32(10.0) ** g.uniform(-8, 3, 6).astype(np.float32):
+        got = oracle.dequant_scaled(codes[fin], float(s), fmt)
+        ref = (torch.from_numpy(table[fin].astype(np.float32)) * torch.tensor(float(s), dtype=torch.float32))
+        assert np.array_equal(got, ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
 def test_ffs_outlier_example():
     rows, table = read_golden("ffs_outlier_example.txt")
     x = np.array([float(r[0]) for r in table], np.float32)
