@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8.so")
 SOURCES = ["api.cu", "quantize.cu", "gemm_sm100.cu", "decode_sm100.cu", "wo_sm100.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "gemm_common.cuh", "kernels.h", "ptx.cuh"]
-PUBLIC_HEADER = os.path.join(os.path.dirname(HERE), "include", "fp8.h")
+PUBLIC_HEADERS = [os.path.join(os.path.dirname(HERE), "include", h) for h in ("fp8.h", "fp8_testing.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -31,7 +31,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [PUBLIC_HEADER]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + PUBLIC_HEADERS
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -6,6 +6,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "../../include/fp8_testing.h"
 
 using namespace fp8b;
 
@@ -208,6 +209,8 @@ const char* fp8_status_string(int32_t s) {
 }
 
 int32_t fp8_device_check(void) { return device_gate(); }
+
+void fp8_testing_set_wait_limit_ns(uint64_t ns) { set_wait_limit_ns(ns); }
 
 size_t fp8_workspace_size(int32_t which, int64_t M, int64_t N, int64_t K, int32_t mode) {
     (void)N;

@@ -149,15 +149,21 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     for (int32_t b = 0; b < kbs; ++b)
                         ptx::tma_load_2d(st + x_off + b * d.nt * BK, &tmX, &full[stage], (kb0 + b) * BK, 0);
             };
+            IssuedLoads loads;
             for (int32_t i = 0; i < pre; ++i) issue(i, (uint32_t)i, true, false);   // fresh ring: no waits
             pdl_wait();
-            for (int32_t i = 0; i < pre; ++i) issue(i, (uint32_t)i, false, true);
+            for (int32_t i = 0; i < pre; ++i) {
+                issue(i, (uint32_t)i, false, true);
+                loads.note((uint32_t)i, 0u);
+            }
             uint32_t stage = (uint32_t)(pre % S), phase = (pre == S) ? 1u : 0u;
             for (int32_t i = pre; i < total; ++i) {
-                if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) break;
+                if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns)) break;
                 issue(i, stage, true, true);
+                loads.note(stage, phase);
                 if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
             }
+            loads.drain(full, p.status);      // loads in flight after an abort
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer: D[n, m] += W X^T
@@ -166,11 +172,11 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t s0 = ptx::smem_u32(stages);
         for (int32_t j = 0; j < range.nch && ok; ++j) {
             const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
-            if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
             ptx::tc_fence_after();
             for (int32_t kc = 0; kc < nkc; ++kc) {
                 const int32_t kbs = min(d.kbs, p.num_kb - kc * d.kbs);
-                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 ptx::tc_fence_after();
                 if (lane == 0) {
                     const uint32_t st = s0 + stage * d.stage_bytes;
@@ -192,9 +198,9 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             __syncwarp();
             ++acc_it;
         }
-        if (lane == 0) {
+        if (lane == 0) {                      // issued MMAs finish before TMEM is freed
             ptx::mma_commit(teardown);
-            wait_bounded(teardown, 0, abort_flag, p.status);
+            wait_drain(teardown, 0, p.status);
         }
         __syncwarp();
     } else {
@@ -215,7 +221,7 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             int32_t n0, w;
             decode_chunk(range, j, n0, w);
             const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
-            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) break;
+            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns)) break;
             ptx::tc_fence_after();
             const int32_t r = quarter * 32 + lane;                 // row of the chunk
             const int32_t n = n0 + r;

@@ -21,7 +21,13 @@ constexpr int UMMA_K = 32;          // K per tcgen05.mma for 8-bit operands
 constexpr int STAGES = 4;
 constexpr uint32_t A_STAGE_BYTES = BM * BK;   // 16 KB
 constexpr uint32_t B_STAGE_BYTES = BN * BK;   // 32 KB
-constexpr uint64_t WAIT_TIMEOUT_NS = 4000000000ull;   // 4 s
+constexpr uint64_t WAIT_TIMEOUT_NS = 4000000000ull;   // 4 s: default limit of a pipeline wait
+constexpr uint64_t DRAIN_LIMIT_NS = 2000000000ull;    // 2 s: limit of a wait for hardware completion
+
+// Limit of the pipeline waits of the kernels launched next from this process (0: the
+// default WAIT_TIMEOUT_NS).  Set only through the testing entry point that exercises
+// the failure path (fp8_testing_set_wait_limit_ns); read when a launch is prepared.
+uint64_t wait_limit_ns();
 
 struct GemmParams {
     int32_t M, N, K;
@@ -57,11 +63,14 @@ struct GemmParams {
     // launched as the programmatic dependent of the kernel that produced A (and only A);
     // every kernel waits (pdl_wait) before it reads A or the scales
     int32_t pdl;
+    uint64_t wait_ns;       // limit of each pipeline wait (wait_limit_ns() at launch)
 };
 
 // ---------------------------------------------------------------- bounded waits
+// A pipeline wait: gives up when another warp of the CTA has raised the abort flag, or
+// after limit_ns, when it raises the flag itself and reports FP8_ERR_TIMEOUT.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
-                                             int32_t* status) {
+                                             int32_t* status, uint64_t limit_ns) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer();
     while (true) {
@@ -69,13 +78,47 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
         for (int i = 0; i < 32; ++i)
             if (ptx::mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+        if (ptx::globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             report_status(status, FP8_ERR_TIMEOUT);
             return false;
         }
     }
 }
+
+// A wait for a phase that the hardware completes by itself (the bytes of a TMA load
+// this CTA issued, a tcgen05.commit of MMAs it issued).  Unlike a pipeline wait it
+// ignores the abort flag: an aborting CTA must not release its shared memory or its
+// TMEM while a copy or an MMA still writes or reads them.  Still bounded (2 s), so
+// that nothing can hold the GPU; on expiry it reports FP8_ERR_TIMEOUT and returns.
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, int32_t* status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer() - t0 > DRAIN_LIMIT_NS) {
+            report_status(status, FP8_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// The TMA loads a producer thread has issued: per ring stage, whether any was issued
+// and the phase parity of the last one.  The last load of a stage completes the
+// phase of that parity on the stage's full barrier (earlier ones completed before the
+// stage was refilled), so waiting for those phases waits for every load in flight.
+struct IssuedLoads {
+    uint32_t issued = 0, parity = 0;
+    __device__ __forceinline__ void note(uint32_t stage, uint32_t phase) {
+        issued |= 1u << stage;
+        parity = (parity & ~(1u << stage)) | ((phase & 1u) << stage);
+    }
+    // Before the CTA may exit: every issued load has landed.
+    __device__ __forceinline__ void drain(uint64_t* full, int32_t* status) const {
+        for (uint32_t s = 0; s < 32; ++s)
+            if ((issued >> s) & 1u) wait_drain(&full[s], (parity >> s) & 1u, status);
+    }
+};
 
 // Write 32 bf16 (16 packed words) of one row into a 32x32 staging tile laid out
 // for the 64-byte TMA swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r>>1)&3).

@@ -24,7 +24,9 @@
 //   MX        MXFP8: E8M0 scales for every 32 K of each row/column are copied into
 //             TMEM and applied by the tensor core itself.
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA raises an abort
-// flag, reports FP8_ERR_TIMEOUT in dev_status, drains and frees TMEM, and exits.
+// flag and reports FP8_ERR_TIMEOUT in dev_status; before it frees TMEM and exits it
+// waits (bounded) for the TMA loads and the MMAs it has already issued.
+#include <atomic>
 #include <cstdio>
 
 #include "gemm_common.cuh"
@@ -147,17 +149,23 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             pdl_wait();                       // A may come from the kernel just before
             uint32_t stage = 0, phase = 0;
             bool ok = true;
+            IssuedLoads loads;
             for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int32_t mb, nb;
                 tile_coords(p, t, mb, nb);
                 for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&full[stage], A_STAGE_BYTES + B_STAGE_BYTES);
                     ptx::tma_load_2d(sA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, mb * BM);
                     ptx::tma_load_2d(sB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+                    loads.note(stage, phase);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
+            // after an abort, loads may still be landing in the ring: wait for all of them
+            // (MX: a stage whose scale factors never came never completes; its wait runs
+            // out after the drain limit, long after the copy itself has landed)
+            loads.drain(full, p.status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -168,16 +176,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             if (V != V_BLOCK) {
                 const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
-                if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 ptx::tc_fence_after();
             }
             for (int32_t kb = 0; kb < p.num_kb; ++kb) {
                 if (V == V_BLOCK) {
                     const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
-                    if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::tc_fence_after();
                 }
-                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (acc_it % C::ACC_BUFS) * BN;
                 if (lane == 0) {
@@ -216,10 +224,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 ++acc_it;
             }
         }
-        // all issued tcgen05 work must finish before TMEM is released
+        // all issued tcgen05 work must finish before TMEM and shared memory are released,
+        // on the normal path and after an abort alike
         if (lane == 0) {
             ptx::mma_commit(teardown);
-            wait_bounded(teardown, 0, abort_flag, p.status);
+            wait_drain(teardown, 0, p.status);
         }
         __syncwarp();
     } else if (V == V_MX && warp == 2) {
@@ -237,7 +246,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const bool vec16 = (kg % 16) == 0 && ((reinterpret_cast<uintptr_t>(p.sfa) | reinterpret_cast<uintptr_t>(p.sfb)) & 15u) == 0;
         auto put_stage = [&](uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t w4, uint32_t w5,
                              uint32_t w6, uint32_t w7, uint32_t w8, uint32_t w9, uint32_t w10, uint32_t w11) -> bool {
-            if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) return false;
+            if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns)) return false;
             uint8_t* dst = sSF + stage * SF_STAGE_BYTES;
             *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(w0, w1, w2, w3);
             *reinterpret_cast<uint4*>(dst + 512 + lane * 16) = make_uint4(w4, w5, w6, w7);
@@ -334,7 +343,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const int32_t y_row0 = mb * BM + quarter * 32;
             if (V == V_ROWSCALE) {
                 const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
-                if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const float sx = row < p.M ? __ldg(p.sa + (int64_t)row * p.sa_stride) : 0.0f;
 #pragma unroll 1
@@ -371,7 +380,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 // one promotion step: P_kb (in TMEM buffer `buf`) * s added into acc
                 auto promote = [&](float s) -> bool {
                     const uint32_t buf = acc_it % C::ACC_BUFS, use = acc_it / C::ACC_BUFS;
-                    if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) return false;
+                    if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns)) return false;
                     ptx::tc_fence_after();
                     const float2 s2 = make_float2(s, s);
 #pragma unroll
@@ -447,7 +456,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
                 }
             } else {  // V_MX: drain the single accumulator into registers, then store
-                if (!wait_bounded(&tfull[0], acc_it & 1u, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&tfull[0], acc_it & 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 ptx::tc_fence_after();
                 uint32_t r[4][32];
 #pragma unroll
@@ -583,17 +592,20 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             pdl_wait();                       // A may come from the kernel just before
             uint32_t stage = 0, phase = 0;
             bool ok = true;
+            IssuedLoads loads;
             for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
                 int32_t mb, nb;
                 tile_coords(p, t, mb, nb);
                 for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&full[stage], 2 * P_HALF_BYTES);
                     ptx::tma_load_2d(sA + stage * P_HALF_BYTES, &tmA, &full[stage], kb * BK, mb * P_BM + (int32_t)rank * 128);
                     ptx::tma_load_2d(sB + stage * P_HALF_BYTES, &tmB, &full[stage], kb * BK, nb * BN + (int32_t)rank * 128);
+                    loads.note(stage, phase);
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
+            loads.drain(full, p.status);      // this CTA's loads in flight, after an abort
         }
     } else if (warp == 2) {
         // ------------------------------------------------ relay (both CTAs)
@@ -602,7 +614,7 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             bool ok = true;
             for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
                 for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::mbar_arrive_cluster(&ready[stage], 0);
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -616,10 +628,10 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const uint32_t sA0 = ptx::smem_u32(sA), sB0 = ptx::smem_u32(sB);
             for (int32_t t = cluster; t < num_tiles && ok; t += nclusters) {
                 const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
-                if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 ptx::tc_fence_after();
                 for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(&ready[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&ready[stage], phase, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::tc_fence_after();
                     if (lane == 0) {
 #pragma unroll
@@ -638,9 +650,11 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 __syncwarp();
                 ++acc_it;
             }
+            // the pair's MMAs read both CTAs' shared memory: they finish before either CTA
+            // reaches the closing cluster barrier
             if (lane == 0) {
                 ptx::mma_commit_pair(teardown, 0x1);
-                wait_bounded(teardown, 0, abort_flag, p.status);
+                wait_drain(teardown, 0, p.status);
             }
             __syncwarp();
         }
@@ -661,7 +675,7 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const int32_t y_row0 = mb * P_BM + (int32_t)rank * 128 + quarter * 32;
             const int32_t row = y_row0 + lane;
             const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
-            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) { ok = false; break; }
+            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
             ptx::tc_fence_after();
             const float sx = row < p.M ? __ldg(p.sa + (int64_t)row * p.sa_stride) : 0.0f;
 #pragma unroll 1
@@ -700,6 +714,15 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 }
 
 // ================================================================ host side
+static std::atomic<uint64_t> g_wait_limit_ns{0};
+
+void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns, std::memory_order_relaxed); }
+
+uint64_t wait_limit_ns() {
+    const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+    return v != 0 ? v : WAIT_TIMEOUT_NS;
+}
+
 template <int V, bool EXT>
 static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaStream_t st) {
     CUtensorMap ta, tb, ty;
@@ -838,6 +861,7 @@ static void set_epilogue(const GemmArgs& g, GemmParams& p) {
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
     GemmParams p{};
+    p.wait_ns = wait_limit_ns();
     p.M = (int32_t)g.M;
     p.N = (int32_t)g.N;
     p.K = (int32_t)g.K;
@@ -923,6 +947,7 @@ __global__ void __launch_bounds__(256) epi_zero_k_kernel(const GemmParams p) {
 
 cudaError_t launch_zero_k_epilogue(const GemmArgs& g, cudaStream_t st) {
     GemmParams p{};
+    p.wait_ns = wait_limit_ns();
     p.M = (int32_t)g.M;
     p.N = (int32_t)g.N;
     p.K = 0;

@@ -60,6 +60,10 @@ struct GemmArgs {
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
 
+// Limit of every pipeline wait in the kernels launched from now on (0: the default);
+// only the testing entry point fp8_testing_set_wait_limit_ns calls this.
+void set_wait_limit_ns(uint64_t ns);
+
 struct WoArgs {              // weight-only FP8 linear (wo_sm100.cu)
     const uint16_t* x;       // bf16 [M, K], row stride ldx
     int64_t ldx;

@@ -171,10 +171,12 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
     }
     if (SRC != SRC_GIVEN) src = block_max_u32(src, red);
     float amax;
+    bool finite_in = true;     // step 0 of a delayed history records only a finite amax
     if (SRC == SRC_PARTIALS) {
         if (src >= 0x7F80u) {
             if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) report_status(status, FP8_ERR_NONFINITE);
             src = 0x7F7Fu;     // keep the scale finite; outputs are unspecified then
+            finite_in = false;
         }
         amax = bf16bits_to_float(src);
     } else if (SRC == SRC_RING) {
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
     const DivScale op{scale_from_amax<FMT>(amax)};
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         scale_out[0] = op.s;
-        if (SRC == SRC_PARTIALS && ring != nullptr) ring[slot] = amax;
+        if (SRC == SRC_PARTIALS && ring != nullptr && finite_in) ring[slot] = amax;
     }
     constexpr bool CHECK = SRC != SRC_PARTIALS;   // inputs not already scanned by phase 1
     // ---- the cast
@@ -230,10 +232,11 @@ __global__ void __launch_bounds__(QT) cast_tensor_kernel(
             const uint32_t total = gridDim.x * gridDim.y;
             uint32_t t = atomicAdd(ticket, 1u);
             if (t == total - 1) {
-                // every CTA has read the ring (they all did so before taking a ticket)
+                // every CTA has read the ring (they all did so before taking a ticket);
+                // a step that saw a NaN/Inf records nothing: its slot keeps the old amax
                 __threadfence();
                 uint32_t a_t = atomicOr(reinterpret_cast<uint32_t*>(pending), 0u);
-                ring[slot] = __uint_as_float(a_t);
+                if (a_t < 0x7F800000u) ring[slot] = __uint_as_float(a_t);
                 *reinterpret_cast<volatile uint32_t*>(pending) = 0u;
                 *reinterpret_cast<volatile uint32_t*>(ticket) = 0u;
             }
@@ -657,10 +660,12 @@ __global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(
     }
     if (KIND != RQ_GIVEN) src = block_max_u32(src, red);
     float amax;
+    bool finite_in = true;     // step 0 of a delayed history records only a finite amax
     if (KIND == RQ_CAST) {
         if (src >= 0x7F80u) {
             if (blockIdx.x == 0 && threadIdx.x == 0) report_status(p.status, FP8_ERR_NONFINITE);
             src = 0x7F7Fu;
+            finite_in = false;
         }
         amax = bf16bits_to_float(src);
     } else if (KIND == RQ_DELAYED) {
@@ -677,7 +682,7 @@ __global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(
     const uint32_t fast_lim = min(__float_as_uint(__fmul_rn(s, 1.7014118e38f)) >> 16, 0x7F7Fu);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         reinterpret_cast<float*>(p.scale)[0] = s;
-        if (KIND == RQ_CAST && p.ring != nullptr) p.ring[p.slot] = amax;
+        if (KIND == RQ_CAST && p.ring != nullptr && finite_in) p.ring[p.slot] = amax;
     }
     const int64_t nvec = p.n / VEC;
     const int64_t stride = (int64_t)gridDim.x * QT;
@@ -717,10 +722,12 @@ __global__ void __launch_bounds__(QT, KIND == RQ_CAST ? 6 : 5) rq_tensor_kernel(
             __threadfence();
             const uint32_t ticket = atomicAdd(p.ticket, 1u);
             if (ticket == gridDim.x - 1) {
-                // every CTA read the ring before taking its ticket
+                // every CTA read the ring before taking its ticket; a step that saw a
+                // NaN/Inf records nothing (its slot keeps the old amax), so one bad step
+                // cannot set the scale of the next h steps
                 __threadfence();
                 const uint32_t a_t = atomicOr(reinterpret_cast<uint32_t*>(p.pending), 0u);
-                p.ring[p.slot] = __uint_as_float(a_t);
+                if (a_t < 0x7F800000u) p.ring[p.slot] = __uint_as_float(a_t);
                 *reinterpret_cast<volatile uint32_t*>(p.pending) = 0u;
                 *reinterpret_cast<volatile uint32_t*>(p.ticket) = 0u;
             }
@@ -749,7 +756,8 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const
         m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(v[j]));
     }
     uint32_t m = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
-    if (m >= 0x7F80u) {
+    const bool finite_in = m < 0x7F80u;
+    if (!finite_in) {
         if (threadIdx.x == 0) report_status(p.status, FP8_ERR_NONFINITE);
         m = 0x7F7Fu;
     }
@@ -757,7 +765,7 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const
     const RcpScale op = rcp_scale_from_amax_bits<FMT>(m);
     if (threadIdx.x == 0) {
         reinterpret_cast<float*>(p.scale)[0] = op.s;
-        if (p.ring != nullptr) p.ring[p.slot] = amax;          // delayed scaling, step 0
+        if (p.ring != nullptr && finite_in) p.ring[p.slot] = amax;   // delayed scaling, step 0
     }
 #pragma unroll
     for (int j = 0; j < SMALL_VPT; ++j) {

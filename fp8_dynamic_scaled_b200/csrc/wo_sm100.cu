@@ -148,13 +148,14 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             bool ok = true;
+            IssuedLoads loads;
             for (int32_t j = 0; j < range.nch && ok; ++j) {
                 int32_t n0, w;
                 wo_chunk(range, j, n0, w);
                 for (int32_t kc = 0; kc < nkc; ++kc) {
                     const int32_t kb0 = kc * WO_KBS;
                     const int32_t kbs = min(WO_KBS, p.num_kb - kb0);
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     uint8_t* st = stages + stage * d.stage_bytes;
                     ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)kbs * ((uint32_t)w * BK + 2 * x_half));
                     for (int32_t r = 0; r < w;) {
@@ -168,9 +169,11 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                         for (int h = 0; h < 2; ++h)
                             ptx::tma_load_2d(st + x_off + (2 * b + h) * x_half, &tmX, &full[stage],
                                              (kb0 + b) * BK + h * 64, 0);
+                    loads.note(stage, phase);
                     if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
                 }
             }
+            loads.drain(full, p.status);      // loads in flight after an abort
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer: D[n, m] += W_bf16 X^T
@@ -179,15 +182,15 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         const uint32_t s0 = ptx::smem_u32(stages), r0 = ptx::smem_u32(ring);
         for (int32_t j = 0; j < range.nch && ok; ++j) {
             const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
-            if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
             ptx::tc_fence_after();
             for (int32_t kc = 0; kc < nkc && ok; ++kc) {
                 const int32_t kbs = min(WO_KBS, p.num_kb - kc * WO_KBS);
-                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 const uint32_t sx = s0 + stage * d.stage_bytes + x_off;
                 for (int32_t hb = 0; hb < 2 * kbs; ++hb) {
                     const uint32_t t = conv_it % WO_SLOTS, tu = conv_it / WO_SLOTS;
-                    if (!wait_bounded(&bfull[t], tu & 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&bfull[t], tu & 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::tc_fence_after();
                     if (lane == 0) {
 #pragma unroll
@@ -211,9 +214,9 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             __syncwarp();
             ++acc_it;
         }
-        if (lane == 0) {
+        if (lane == 0) {                      // issued MMAs finish before TMEM is freed
             ptx::mma_commit(teardown);
-            wait_bounded(teardown, 0, abort_flag, p.status);
+            wait_drain(teardown, 0, p.status);
         }
         __syncwarp();
     } else if (warp < WO_FIRST_EPI) {
@@ -227,11 +230,11 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         for (int32_t j = 0; j < range.nch && ok; ++j) {
             for (int32_t kc = 0; kc < nkc && ok; ++kc) {
                 const int32_t kbs = min(WO_KBS, p.num_kb - kc * WO_KBS);
-                if (!wait_bounded(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_bounded(&full[stage], phase, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                 const uint8_t* w8 = stages + stage * d.stage_bytes;
                 for (int32_t hb = 0; hb < 2 * kbs; ++hb) {
                     const uint32_t t = conv_it % WO_SLOTS, tu = conv_it / WO_SLOTS;
-                    if (!wait_bounded(&bempty[t], (tu & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_bounded(&bempty[t], (tu & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     const int b = hb >> 1, h = hb & 1;
                     const uint8_t* src = w8 + b * WO_W8_BYTES + row * 128;
                     uint8_t* dst = ring + t * WO_HALF_BYTES + row * 128;
@@ -261,7 +264,7 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             int32_t n0, w;
             wo_chunk(range, j, n0, w);
             const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
-            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status)) break;
+            if (!wait_bounded(&tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns)) break;
             ptx::tc_fence_after();
             const int32_t r = quarter * 32 + lane;
             const int32_t n = n0 + r;
@@ -297,6 +300,7 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 template <int WFMT>
 static cudaError_t launch_wo_t(const WoArgs& g, cudaStream_t st) {
     GemmParams p{};
+    p.wait_ns = wait_limit_ns();
     p.M = (int32_t)g.M;
     p.N = (int32_t)g.N;
     p.K = (int32_t)g.K;

@@ -95,8 +95,11 @@ typedef enum {
  *   ticket_dev   one device uint32, zero before step 0 (CTA arrival counter).
  * Step 0 has no history and uses current per-tensor scaling; step t >= 1 uses
  * s_t = max(max(ring), 1e-12f) / F_max.  After the step, ring[t mod h] holds the
- * raw amax of X_t, and pending/ticket are back to zero.  Two steps on the same
- * history must be stream-ordered.
+ * raw amax of X_t, and pending/ticket are back to zero.  A step whose input holds a
+ * NaN/Inf (FP8_ERR_NONFINITE in dev_status; that step's outputs are unspecified)
+ * records nothing: ring[t mod h] keeps its previous value, so the bad step does
+ * not set the scale of the h steps after it, and step still advances.  Two steps
+ * on the same history must be stream-ordered.
  */
 typedef struct {
     float* ring_dev;
@@ -316,7 +319,9 @@ FP8_API int32_t fp8_weight_only_linear(const void* x_dev, int64_t M, int64_t K, 
  *     inputs return FP8_ERR_WORKSPACE and enqueue nothing.
  *   - The first call on each device looks up the scratch's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *     before any stream capture begins.  The address is kept for the life of the
+ *     process: a cudaDeviceReset (or anything else that unloads the library's
+ *     device code) after the first call is not supported.
  *   - All calls share the one scratch array, which keeps the last call's
  *     contents (nothing in it needs to start at zero).  Calls whose work can
  *     overlap on the GPU -- different streams, or unordered host threads -- race

@@ -33,7 +33,7 @@ def build(force: bool = False) -> str:
             and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
         return _LIB_PATH
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+    cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-pthread",
            "-shared", "-o", tmp, _SRC, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, _LIB_PATH)
@@ -73,6 +73,8 @@ def _load():
     lib.orc_quant_scaled_array.argtypes = [P, I64, F, I32, P]
     lib.orc_dequant_scaled_array.restype = None
     lib.orc_dequant_scaled_array.argtypes = [P, I64, F, I32, P]
+    lib.orc_set_threads.restype, lib.orc_set_threads.argtypes = None, [I32]
+    lib.orc_get_threads.restype, lib.orc_get_threads.argtypes = I32, []
     _lib = lib
     return lib
 
@@ -86,6 +88,31 @@ def _ptr(a: np.ndarray | None):
 
 class OracleError(RuntimeError):
     pass
+
+
+def set_threads(n: int) -> None:
+    """Threads the oracle's array-wide functions use (rows, row blocks or output points
+    split into contiguous ranges; the results do not depend on the count).  Default 1."""
+    _load().orc_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_load().orc_get_threads())
+
+
+class threads:
+    """Context manager: run the oracle on `n` threads inside the block."""
+
+    def __init__(self, n: int):
+        self.n = int(n)
+
+    def __enter__(self):
+        self.prev = get_threads()
+        set_threads(self.n)
+        return self
+
+    def __exit__(self, *exc):
+        set_threads(self.prev)
 
 
 def fmax(fmt: int) -> float:
@@ -264,6 +291,46 @@ def gemm_ref_points(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b, pm, pn):
         raise OracleError("orc_gemm_ref_points failed")
     y[order] = ys
     bound[order] = bs
+    return y, bound
+
+
+def _dequant_rows_f64(codes, scale, mode: int, fmt: int, rows: np.ndarray) -> np.ndarray:
+    """S(r, k) * decode(codes[r, k]) in fp64 for the given rows r (the scale that covers
+    each element, in the layouts of ``quantize``)."""
+    codes = np.asarray(codes, np.uint8)
+    K = codes.shape[1]
+    v = decode_table(fmt)[codes[rows]]
+    s = np.asarray(scale)
+    if mode in (TENSOR, DELAYED):
+        return v * np.float64(s.reshape(-1)[0])
+    if mode == ROW:
+        return v * s.reshape(-1)[rows].astype(np.float64)[:, None]
+    if mode == BLOCK_1x128:
+        return v * np.repeat(s[rows].astype(np.float64), 128, axis=1)[:, :K]
+    if mode == BLOCK_128x128:
+        return v * np.repeat(s[rows // 128].astype(np.float64), 128, axis=1)[:, :K]
+    if mode == MX32:
+        return v * np.repeat(np.exp2(s[rows].astype(np.float64) - 127.0), 32, axis=1)
+    raise ValueError(mode)
+
+
+def gemm_ref_rows(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b, rows, chunk: int = 2048):
+    """fp64 reference of whole output rows: y[i, n] = sum_k A_deq[rows[i], k] B_deq[n, k]
+    and the bound sum_k |same product| ([FFS] "一次 FP8 GEMM 的完整精度契约"), for bands of
+    rows of a large GEMM.  The operands are dequantised exactly in fp64 (a code times a
+    power of two or an fp32 scale) and the sums run through NumPy's fp64 matmul (a
+    library step), B in chunks of `chunk` rows to bound the memory."""
+    rows = np.asarray(rows, np.int64)
+    ad = _dequant_rows_f64(a, sa, a_mode, fmt_a, rows)
+    aa = np.abs(ad)
+    N = np.asarray(b).shape[0]
+    y = np.empty((rows.size, N), np.float64)
+    bound = np.empty((rows.size, N), np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        bd = _dequant_rows_f64(b, sb, b_mode, fmt_b, np.arange(n0, n1))
+        y[:, n0:n1] = ad @ bd.T
+        bound[:, n0:n1] = aa @ np.abs(bd).T
     return y, bound
 
 

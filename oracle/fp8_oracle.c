@@ -32,13 +32,17 @@
  *  - negative values that round to zero keep their sign (code 0x80);
  *  - MX32: e = clamp(floor(log2 amax) - 8, -127, 127), byte = e + 127, amax = 0 -> e = -127;
  *  - delayed: step 0 uses the current amax, later steps the max over the ring,
- *    and amax_t of the raw input is written to ring[t mod h] after use.
+ *    and amax_t of the raw input is written to ring[t mod h] after use; a step
+ *    whose input holds a NaN/Inf is refused and writes nothing to the ring.
+ *  - threads: rows (row blocks, output points) may be split over threads; every
+ *    element is computed by the same code, so the results do not depend on it.
  *
  * Parity status: every function here is pinned (tests/test_oracle_pins.py and
  * tests/test_oracle_epilogue_pins.py: printed examples under tests/golden, closed
  * forms, exact integer arithmetic, brute force); none is "parity unpinned".
  */
 #include <math.h>
+#include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -265,6 +269,65 @@ int64_t orc_scale_count(int mode, int64_t rows, int64_t cols) {
 }
 
 /* ------------------------------------------------------------------ */
+/* Threads.  The array-wide entry points split their rows (row blocks,  */
+/* output points) into contiguous ranges, one per thread.  Every        */
+/* element is still produced by the same code, and a maximum or a count */
+/* does not depend on how the ranges are combined, so the results are   */
+/* the same for every thread count.  Default: 1 thread.                 */
+/* ------------------------------------------------------------------ */
+#define ORC_MAX_THREADS 256
+static int g_threads = 1;
+
+void orc_set_threads(int n) { g_threads = n < 1 ? 1 : (n > ORC_MAX_THREADS ? ORC_MAX_THREADS : n); }
+int orc_get_threads(void) { return g_threads; }
+
+typedef void (*orc_range_fn)(void* ctx, int64_t i0, int64_t i1, int part);
+typedef struct {
+    orc_range_fn fn;
+    void* ctx;
+    int64_t i0, i1;
+    int part;
+} orc_job;
+
+static void* orc_job_main(void* p) {
+    orc_job* j = (orc_job*)p;
+    j->fn(j->ctx, j->i0, j->i1, j->part);
+    return NULL;
+}
+
+/* Run fn on [0, n) cut into at most g_threads ranges whose bounds are multiples of
+ * `grain`; range k gets part index k.  Returns the number of ranges. */
+static int orc_parallel(int64_t n, int64_t grain, void* ctx, orc_range_fn fn) {
+    if (n <= 0) return 0;
+    if (grain < 1) grain = 1;
+    int64_t units = (n + grain - 1) / grain;
+    int parts = g_threads;
+    if (parts > units) parts = (int)units;
+    if (parts <= 1) {
+        fn(ctx, 0, n, 0);
+        return 1;
+    }
+    orc_job jobs[ORC_MAX_THREADS];
+    pthread_t th[ORC_MAX_THREADS];
+    int started[ORC_MAX_THREADS];
+    for (int k = 0; k < parts; ++k) {
+        int64_t u0 = units * k / parts, u1 = units * (k + 1) / parts;
+        jobs[k].fn = fn;
+        jobs[k].ctx = ctx;
+        jobs[k].i0 = u0 * grain;
+        jobs[k].i1 = u1 * grain < n ? u1 * grain : n;
+        jobs[k].part = k;
+    }
+    for (int k = 1; k < parts; ++k) started[k] = pthread_create(&th[k], NULL, orc_job_main, &jobs[k]) == 0;
+    fn(ctx, jobs[0].i0, jobs[0].i1, 0);
+    for (int k = 1; k < parts; ++k) {
+        if (started[k]) pthread_join(th[k], NULL);
+        else fn(ctx, jobs[k].i0, jobs[k].i1, k);   /* no thread: run the range here */
+    }
+    return parts;
+}
+
+/* ------------------------------------------------------------------ */
 /* amax over a rectangular region of a bf16 matrix.                    */
 /* ------------------------------------------------------------------ */
 static float amax_region(const uint16_t* x, int64_t ld, int64_t r0, int64_t r1,
@@ -278,12 +341,118 @@ static float amax_region(const uint16_t* x, int64_t ld, int64_t r0, int64_t r1,
     return m;
 }
 
-/* Returns 0 on success, 1 on a non-finite input, 2 on a bad argument. */
-static int check_finite(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld) {
-    for (int64_t r = 0; r < rows; ++r)
-        for (int64_t c = 0; c < cols; ++c)
-            if (!isfinite(bf16_to_f32(x[r * ld + c]))) return 1;
+/* State shared by the row-range workers of orc_quantize / orc_delayed_step. */
+typedef struct {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    int fmt;
+    uint8_t* q;
+    void* scale;
+    uint16_t* dequant;
+    float s;                              /* per-tensor scale of the cast */
+    float amax_part[ORC_MAX_THREADS];     /* per-range amax */
+    int64_t sat_part[ORC_MAX_THREADS];    /* per-range count of |x / s| > F_max */
+    int bad_part[ORC_MAX_THREADS];        /* per-range: a non-finite element seen */
+} qjob;
+
+static void finite_rows(void* c, int64_t r0, int64_t r1, int part) {
+    qjob* j = (qjob*)c;
+    int bad = 0;
+    for (int64_t r = r0; r < r1 && !bad; ++r)
+        for (int64_t k = 0; k < j->cols; ++k)
+            if (!isfinite(bf16_to_f32(j->x[r * j->ld + k]))) { bad = 1; break; }
+    j->bad_part[part] = bad;
+}
+
+/* 1 when any element of x is NaN or Inf. */
+static int check_finite(qjob* j) {
+    int parts = orc_parallel(j->rows, 1, j, finite_rows);
+    for (int k = 0; k < parts; ++k)
+        if (j->bad_part[k]) return 1;
     return 0;
+}
+
+static void amax_rows(void* c, int64_t r0, int64_t r1, int part) {
+    qjob* j = (qjob*)c;
+    j->amax_part[part] = amax_region(j->x, j->ld, r0, r1, 0, j->cols);
+}
+
+/* a_max over the whole tensor: the maximum of the ranges' maxima. */
+static float amax_all(qjob* j) {
+    int parts = orc_parallel(j->rows, 1, j, amax_rows);
+    float m = 0.0f;
+    for (int k = 0; k < parts; ++k)
+        if (j->amax_part[k] > m) m = j->amax_part[k];
+    return m;
+}
+
+/* Cast rows [r0, r1) with the one scale j->s, counting saturated elements. */
+static void cast_rows(void* c, int64_t r0, int64_t r1, int part) {
+    qjob* j = (qjob*)c;
+    int64_t sat_total = 0;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t k = 0; k < j->cols; ++k) {
+            int sat = 0;
+            uint8_t code = quant_one(bf16_to_f32(j->x[r * j->ld + k]), j->s, j->fmt, &sat);
+            sat_total += sat;
+            j->q[r * j->cols + k] = code;
+            if (j->dequant) j->dequant[r * j->cols + k] = dequant_one(code, j->s, j->fmt);
+        }
+    j->sat_part[part] = sat_total;
+}
+
+/* ROW: one scale per row. */
+static void row_rows(void* c, int64_t r0, int64_t r1, int part) {
+    (void)part;
+    qjob* j = (qjob*)c;
+    for (int64_t r = r0; r < r1; ++r) {
+        float s = orc_scale_from_amax(amax_region(j->x, j->ld, r, r + 1, 0, j->cols), j->fmt);
+        ((float*)j->scale)[r] = s;
+        for (int64_t k = 0; k < j->cols; ++k) {
+            uint8_t code = quant_one(bf16_to_f32(j->x[r * j->ld + k]), s, j->fmt, NULL);
+            j->q[r * j->cols + k] = code;
+            if (j->dequant) j->dequant[r * j->cols + k] = dequant_one(code, s, j->fmt);
+        }
+    }
+}
+
+/* BLOCK_1x128 (bh = 1) and BLOCK_128x128 (bh = 128): one scale per bh x 128 block
+ * (ragged blocks at the right and bottom edges); i0..i1 index block rows. */
+static void block_rows(qjob* j, int64_t bh, int64_t br0, int64_t br1) {
+    int64_t nbc = cdiv(j->cols, 128);
+    for (int64_t br = br0; br < br1; ++br)
+        for (int64_t bc = 0; bc < nbc; ++bc) {
+            int64_t r0 = br * bh, r1 = r0 + bh < j->rows ? r0 + bh : j->rows;
+            int64_t c0 = bc * 128, c1 = c0 + 128 < j->cols ? c0 + 128 : j->cols;
+            float s = orc_scale_from_amax(amax_region(j->x, j->ld, r0, r1, c0, c1), j->fmt);
+            ((float*)j->scale)[br * nbc + bc] = s;
+            for (int64_t r = r0; r < r1; ++r)
+                for (int64_t k = c0; k < c1; ++k) {
+                    uint8_t code = quant_one(bf16_to_f32(j->x[r * j->ld + k]), s, j->fmt, NULL);
+                    j->q[r * j->cols + k] = code;
+                    if (j->dequant) j->dequant[r * j->cols + k] = dequant_one(code, s, j->fmt);
+                }
+        }
+}
+static void block1_rows(void* c, int64_t i0, int64_t i1, int part) { (void)part; block_rows((qjob*)c, 1, i0, i1); }
+static void block128_rows(void* c, int64_t i0, int64_t i1, int part) { (void)part; block_rows((qjob*)c, 128, i0, i1); }
+
+/* MX32: one power-of-two scale per 32 consecutive elements of a row. */
+static void mx_rows(void* c, int64_t r0, int64_t r1, int part) {
+    (void)part;
+    qjob* j = (qjob*)c;
+    int64_t ng = j->cols / 32;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t g = 0; g < ng; ++g) {
+            int e = orc_mx_exponent(amax_region(j->x, j->ld, r, r + 1, g * 32, g * 32 + 32));
+            ((uint8_t*)j->scale)[r * ng + g] = (uint8_t)(e + 127);
+            float s2 = (float)ldexp(1.0, e);
+            for (int64_t k = g * 32; k < g * 32 + 32; ++k) {
+                uint8_t code = quant_one_mx(bf16_to_f32(j->x[r * j->ld + k]), e, j->fmt);
+                j->q[r * j->cols + k] = code;
+                if (j->dequant) j->dequant[r * j->cols + k] = dequant_one(code, s2, j->fmt);
+            }
+        }
 }
 
 /*
@@ -294,72 +463,37 @@ static int check_finite(const uint16_t* x, int64_t rows, int64_t cols, int64_t l
  *   scale    TENSOR: float[1]; ROW: float[rows]; BLOCK_1x128: float[rows][ceil(cols/128)];
  *            BLOCK_128x128: float[ceil(rows/128)][ceil(cols/128)]; MX32: uint8[rows][cols/32]
  *   dequant  optional bf16 [rows, cols] (NULL to skip)
- * Returns 0, 1 (non-finite input) or 2 (bad argument).
+ * Returns 0, 1 (non-finite input; nothing is written) or 2 (bad argument).
  */
 int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int mode,
                  uint8_t* q, void* scale, uint16_t* dequant) {
     if (rows < 0 || cols < 0 || ld < cols) return 2;
     if (fmt != ORC_E4M3 && fmt != ORC_E5M2) return 2;
+    if (mode < ORC_TENSOR || mode > ORC_MX32) return 2;
     if (mode == ORC_MX32 && (fmt != ORC_E4M3 || cols % 32 != 0)) return 2;
-    if (check_finite(x, rows, cols, ld)) return 1;
-    if (mode == ORC_TENSOR) {
-        float a = amax_region(x, ld, 0, rows, 0, cols);
-        float s = orc_scale_from_amax(a, fmt);
-        ((float*)scale)[0] = s;
-        for (int64_t r = 0; r < rows; ++r)
-            for (int64_t c = 0; c < cols; ++c) {
-                uint8_t code = quant_one(bf16_to_f32(x[r * ld + c]), s, fmt, NULL);
-                q[r * cols + c] = code;
-                if (dequant) dequant[r * cols + c] = dequant_one(code, s, fmt);
-            }
-        return 0;
+    qjob* j = (qjob*)calloc(1, sizeof(qjob));
+    if (!j) return 2;
+    j->x = x; j->rows = rows; j->cols = cols; j->ld = ld; j->fmt = fmt;
+    j->q = q; j->scale = scale; j->dequant = dequant;
+    int rc = 0;
+    if (check_finite(j)) {
+        rc = 1;
+    } else if (mode == ORC_TENSOR) {
+        /* [FFS] "Scale 怎样把 Tensor 塞进 E4M3": a_max over the tensor, one s, then the cast */
+        j->s = orc_scale_from_amax(amax_all(j), fmt);
+        ((float*)scale)[0] = j->s;
+        orc_parallel(rows, 1, j, cast_rows);
+    } else if (mode == ORC_ROW) {
+        orc_parallel(rows, 1, j, row_rows);
+    } else if (mode == ORC_BLOCK_1x128) {
+        orc_parallel(rows, 1, j, block1_rows);
+    } else if (mode == ORC_BLOCK_128x128) {
+        orc_parallel(cdiv(rows, 128), 1, j, block128_rows);
+    } else {
+        orc_parallel(rows, 1, j, mx_rows);
     }
-    if (mode == ORC_ROW) {
-        for (int64_t r = 0; r < rows; ++r) {
-            float s = orc_scale_from_amax(amax_region(x, ld, r, r + 1, 0, cols), fmt);
-            ((float*)scale)[r] = s;
-            for (int64_t c = 0; c < cols; ++c) {
-                uint8_t code = quant_one(bf16_to_f32(x[r * ld + c]), s, fmt, NULL);
-                q[r * cols + c] = code;
-                if (dequant) dequant[r * cols + c] = dequant_one(code, s, fmt);
-            }
-        }
-        return 0;
-    }
-    if (mode == ORC_BLOCK_1x128 || mode == ORC_BLOCK_128x128) {
-        int64_t bh = mode == ORC_BLOCK_1x128 ? 1 : 128;
-        int64_t nbr = cdiv(rows, bh), nbc = cdiv(cols, 128);
-        for (int64_t br = 0; br < nbr; ++br)
-            for (int64_t bc = 0; bc < nbc; ++bc) {
-                int64_t r0 = br * bh, r1 = r0 + bh < rows ? r0 + bh : rows;
-                int64_t c0 = bc * 128, c1 = c0 + 128 < cols ? c0 + 128 : cols;
-                float s = orc_scale_from_amax(amax_region(x, ld, r0, r1, c0, c1), fmt);
-                ((float*)scale)[br * nbc + bc] = s;
-                for (int64_t r = r0; r < r1; ++r)
-                    for (int64_t c = c0; c < c1; ++c) {
-                        uint8_t code = quant_one(bf16_to_f32(x[r * ld + c]), s, fmt, NULL);
-                        q[r * cols + c] = code;
-                        if (dequant) dequant[r * cols + c] = dequant_one(code, s, fmt);
-                    }
-            }
-        return 0;
-    }
-    if (mode == ORC_MX32) {
-        int64_t ng = cols / 32;
-        for (int64_t r = 0; r < rows; ++r)
-            for (int64_t g = 0; g < ng; ++g) {
-                int e = orc_mx_exponent(amax_region(x, ld, r, r + 1, g * 32, g * 32 + 32));
-                ((uint8_t*)scale)[r * ng + g] = (uint8_t)(e + 127);
-                float s2 = (float)ldexp(1.0, e);
-                for (int64_t c = g * 32; c < g * 32 + 32; ++c) {
-                    uint8_t code = quant_one_mx(bf16_to_f32(x[r * ld + c]), e, fmt);
-                    q[r * cols + c] = code;
-                    if (dequant) dequant[r * cols + c] = dequant_one(code, s2, fmt);
-                }
-            }
-        return 0;
-    }
-    return 2;
+    free(j);
+    return rc;
 }
 
 /*
@@ -370,14 +504,26 @@ int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int 
  *   After quantizing, ring[t mod len] <- amax_t (raw amax of this step's input).
  *   *saturated receives the number of elements with |x / s_t| > F_max.
  *   *scale_out receives s_t.
+ * A step whose input holds a NaN or Inf is refused (returns 1) and records nothing:
+ * ring[t mod len] keeps its value, so that one bad step cannot set the scale of the
+ * next len steps ([FFS] "数值验证看什么": non-finite values are monitored; a
+ * history is only a window of the amax of valid steps).  The caller still counts
+ * the step (the next one is t + 1).
  */
 int orc_delayed_step(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int fmt,
                      float* ring, int32_t len, int64_t t, uint8_t* q, float* scale_out,
                      uint16_t* dequant, int64_t* saturated) {
     if (rows < 0 || cols < 0 || ld < cols || len <= 0 || t < 0) return 2;
     if (fmt != ORC_E4M3 && fmt != ORC_E5M2) return 2;
-    if (check_finite(x, rows, cols, ld)) return 1;
-    float amax_t = amax_region(x, ld, 0, rows, 0, cols);
+    qjob* j = (qjob*)calloc(1, sizeof(qjob));
+    if (!j) return 2;
+    j->x = x; j->rows = rows; j->cols = cols; j->ld = ld; j->fmt = fmt;
+    j->q = q; j->dequant = dequant;
+    if (check_finite(j)) {
+        free(j);
+        return 1;
+    }
+    float amax_t = amax_all(j);
     float s;
     if (t == 0) {
         s = orc_scale_from_amax(amax_t, fmt);
@@ -386,19 +532,14 @@ int orc_delayed_step(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, 
         for (int32_t i = 0; i < len; ++i) if (ring[i] > h) h = ring[i];
         s = orc_scale_from_amax(h, fmt);
     }
-    int sat = 0;
+    j->s = s;
+    int parts = orc_parallel(rows, 1, j, cast_rows);
     int64_t sat_total = 0;
-    for (int64_t r = 0; r < rows; ++r)
-        for (int64_t c = 0; c < cols; ++c) {
-            sat = 0;
-            uint8_t code = quant_one(bf16_to_f32(x[r * ld + c]), s, fmt, &sat);
-            sat_total += sat;
-            q[r * cols + c] = code;
-            if (dequant) dequant[r * cols + c] = dequant_one(code, s, fmt);
-        }
+    for (int k = 0; k < parts; ++k) sat_total += j->sat_part[k];
     *scale_out = s;
     if (saturated) *saturated = sat_total;
     ring[t % len] = amax_t;
+    free(j);
     return 0;
 }
 
@@ -426,36 +567,85 @@ static void deq_row(const uint8_t* codes, const void* scale, int mode, int fmt, 
         out[k] = scale_at(scale, mode, r, k, K) * orc_decode(codes[r * K + k], fmt);
 }
 
-/* Reference at a list of output points (m[i], n[i]). */
-int orc_gemm_ref_points(const uint8_t* a, const void* sa, int a_mode, int fmt_a,
-                        const uint8_t* b, const void* sb, int b_mode, int fmt_b,
-                        int64_t M, int64_t N, int64_t K,
-                        const int64_t* pm, const int64_t* pn, int64_t npts,
-                        double* y, double* bound) {
+/* Reference at a list of output points (m[i], n[i]); the points are split into
+ * contiguous ranges over the threads (each with its own dequantised rows). */
+typedef struct {
+    const uint8_t *a, *b;
+    const void *sa, *sb;
+    int a_mode, fmt_a, b_mode, fmt_b;
+    int64_t M, N, K;
+    const int64_t *pm, *pn;
+    double *y, *bound;
+    int err_part[ORC_MAX_THREADS];
+} pjob;
+
+static void points_range(void* c, int64_t i0, int64_t i1, int part) {
+    pjob* j = (pjob*)c;
+    int64_t K = j->K;
     double* ra = (double*)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
     double* rb = (double*)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
-    if (!ra || !rb) { free(ra); free(rb); return 2; }
+    j->err_part[part] = 0;
+    if (!ra || !rb) { free(ra); free(rb); j->err_part[part] = 1; return; }
     int64_t cur_m = -1;
-    for (int64_t i = 0; i < npts; ++i) {
-        int64_t m = pm[i], n = pn[i];
-        if (m < 0 || m >= M || n < 0 || n >= N) { free(ra); free(rb); return 2; }
-        if (m != cur_m) { deq_row(a, sa, a_mode, fmt_a, m, K, ra); cur_m = m; }
-        deq_row(b, sb, b_mode, fmt_b, n, K, rb);
+    for (int64_t i = i0; i < i1; ++i) {
+        int64_t m = j->pm[i], n = j->pn[i];
+        if (m < 0 || m >= j->M || n < 0 || n >= j->N) { j->err_part[part] = 1; break; }
+        if (m != cur_m) { deq_row(j->a, j->sa, j->a_mode, j->fmt_a, m, K, ra); cur_m = m; }
+        deq_row(j->b, j->sb, j->b_mode, j->fmt_b, n, K, rb);
         double acc = 0.0, bnd = 0.0;
         for (int64_t k = 0; k < K; ++k) {
             double p = ra[k] * rb[k];
             acc += p;
             bnd += fabs(p);
         }
-        y[i] = acc;
-        bound[i] = bnd;
+        j->y[i] = acc;
+        j->bound[i] = bnd;
     }
     free(ra);
     free(rb);
-    return 0;
 }
 
-/* Full reference for small problems: y and bound are [M, N]. */
+int orc_gemm_ref_points(const uint8_t* a, const void* sa, int a_mode, int fmt_a,
+                        const uint8_t* b, const void* sb, int b_mode, int fmt_b,
+                        int64_t M, int64_t N, int64_t K,
+                        const int64_t* pm, const int64_t* pn, int64_t npts,
+                        double* y, double* bound) {
+    pjob* j = (pjob*)calloc(1, sizeof(pjob));
+    if (!j) return 2;
+    j->a = a; j->b = b; j->sa = sa; j->sb = sb;
+    j->a_mode = a_mode; j->fmt_a = fmt_a; j->b_mode = b_mode; j->fmt_b = fmt_b;
+    j->M = M; j->N = N; j->K = K; j->pm = pm; j->pn = pn; j->y = y; j->bound = bound;
+    int parts = orc_parallel(npts, 1, j, points_range);
+    int rc = 0;
+    for (int k = 0; k < parts; ++k)
+        if (j->err_part[k]) rc = 2;
+    free(j);
+    return rc;
+}
+
+/* Full reference: y and bound are [M, N]; rows of the output split over the threads. */
+typedef struct {
+    const double *da, *db;
+    int64_t N, K;
+    double *y, *bound;
+} fjob;
+
+static void full_rows(void* c, int64_t m0, int64_t m1, int part) {
+    (void)part;
+    fjob* j = (fjob*)c;
+    for (int64_t m = m0; m < m1; ++m)
+        for (int64_t n = 0; n < j->N; ++n) {
+            double acc = 0.0, bnd = 0.0;
+            for (int64_t k = 0; k < j->K; ++k) {
+                double p = j->da[m * j->K + k] * j->db[n * j->K + k];
+                acc += p;
+                bnd += fabs(p);
+            }
+            j->y[m * j->N + n] = acc;
+            j->bound[m * j->N + n] = bnd;
+        }
+}
+
 int orc_gemm_ref_full(const uint8_t* a, const void* sa, int a_mode, int fmt_a,
                       const uint8_t* b, const void* sb, int b_mode, int fmt_b,
                       int64_t M, int64_t N, int64_t K, double* y, double* bound) {
@@ -464,17 +654,8 @@ int orc_gemm_ref_full(const uint8_t* a, const void* sa, int a_mode, int fmt_a,
     if (!da || !db) { free(da); free(db); return 2; }
     for (int64_t m = 0; m < M; ++m) deq_row(a, sa, a_mode, fmt_a, m, K, da + m * K);
     for (int64_t n = 0; n < N; ++n) deq_row(b, sb, b_mode, fmt_b, n, K, db + n * K);
-    for (int64_t m = 0; m < M; ++m)
-        for (int64_t n = 0; n < N; ++n) {
-            double acc = 0.0, bnd = 0.0;
-            for (int64_t k = 0; k < K; ++k) {
-                double p = da[m * K + k] * db[n * K + k];
-                acc += p;
-                bnd += fabs(p);
-            }
-            y[m * N + n] = acc;
-            bound[m * N + n] = bnd;
-        }
+    fjob j = {da, db, N, K, y, bound};
+    orc_parallel(M, 1, &j, full_rows);
     free(da);
     free(db);
     return 0;

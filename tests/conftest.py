@@ -11,6 +11,9 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+    # the oracle splits rows over the host's cores (its results do not depend on the count)
+    import oracle
+    oracle.set_threads(max(1, os.cpu_count() or 1))
 
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")

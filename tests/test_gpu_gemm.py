@@ -172,9 +172,10 @@ def _points(M, N, n, seed):
     return pm, pn
 
 
-def full_size_check(x, w, am, bm, what, npts=3000):
+def full_size_check(x, w, am, bm, what, npts=65536):
     """The whole GPU path (fp8_quantize of X and W, then fp8_scaled_gemm) against the
-    oracle's own quantisation and fp64 GEMM at sampled outputs; every output is also
+    oracle's own quantisation and fp64 GEMM at 65,536 sampled outputs (plus the four
+    corners) and at every output of the first and last 128 rows; every output is also
     checked against an fp32 torch matmul of the oracle's dequantised operands."""
     M, K = x.shape
     N = w.shape[0]
@@ -195,6 +196,10 @@ def full_size_check(x, w, am, bm, what, npts=3000):
     y_ref, bound = oracle.gemm_ref_points(qa_h, sa_h, am, E4M3, qb_h, sb_h, bm, E4M3, pm, pn)
     y_h = to_host_u16(y)
     assert_gemm_close(y_h[pm, pn], y_ref, bound, what + " (oracle points)")
+    band = np.unique(np.concatenate([np.arange(0, min(128, M)), np.arange(max(0, M - 128), M)]))
+    y_band, b_band = oracle.gemm_ref_rows(qa_h, sa_h, am, E4M3, qb_h, sb_h, bm, E4M3, band)
+    assert_gemm_close(y_h[band], y_band, b_band, what + " (oracle, first and last 128 rows)")
+    del y_band, b_band
     # every output against a dequantised fp32 matmul of the oracle's operands (chunked over rows)
     qa, sa = torch.from_numpy(qa_h).cuda(), torch.from_numpy(np.ascontiguousarray(sa_h)).cuda()
     qb, sb = torch.from_numpy(qb_h).cuda(), torch.from_numpy(np.ascontiguousarray(sb_h)).cuda()

@@ -180,13 +180,25 @@ def test_cast_sweep_long_rows_fallback():
 
 
 # ---------------------------------------------------------------- delayed scaling
+def _dev_rows(x_u16, ld=None):
+    """x on the device, with row stride ld (a view into a wider buffer) when given."""
+    rows, cols = x_u16.shape
+    if ld is None or ld == cols:
+        return to_dev_bf16(x_u16)
+    buf = np.zeros((rows, ld), np.uint16)
+    buf[:, :cols] = x_u16
+    return to_dev_bf16(buf)[:, :cols]
+
+
 def run_delayed_sequence(xs, fmt, hist_len=16):
     hist = fp8.History(hist_len)
     ring = np.zeros(hist_len, np.float32)
-    ws = fp8.workspace_for(0, xs[0].shape[0], 0, xs[0].shape[1], fp8.FP8_SCALE_DELAYED)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = None
     for t, x in enumerate(xs):
         rows, cols = x.shape
+        if ws is None:
+            ws = fp8.workspace_for(0, rows, 0, cols, fp8.FP8_SCALE_DELAYED)
         q, s, d = fp8.empty_quant_outputs(rows, cols, fp8.FP8_SCALE_DELAYED, dequant=True)
         fp8.fp8_quantize(to_dev_bf16(x), fmt, fp8.FP8_SCALE_DELAYED, q, s, hist=hist, dequant=d, dev_status=st,
                          workspace=ws)
@@ -253,7 +265,174 @@ def test_mx_operands_full_size():
     check_parity(w, fp8.FP8_E4M3, fp8.FP8_SCALE_MX32, dequant=False, what="W MX32")
 
 
-def test_delayed_full_size_first_steps():
+def test_delayed_full_size_sixteen_steps():
+    """The whole drifting sequence at its full size: 16 steps of X_t [16384, 8192] with
+    std 1 -> 4 and a 16-entry history; scale, codes, dequant and ring bit-exact every step."""
     base = inputs.delayed_base()
-    xs = [inputs.delayed_step_input(t, base=base) for t in range(3)]
+    xs = (inputs.delayed_step_input(t, base=base) for t in range(16))
     run_delayed_sequence(xs, fp8.FP8_E4M3)
+
+
+# ---------------------------------------------------------------- non-finite delayed steps
+@pytest.mark.parametrize("bad_step", [0, 5])
+@pytest.mark.parametrize("bad", [0x7F80, 0xFFC1])          # +Inf, NaN
+@pytest.mark.parametrize("shape,ld", [((64, 256), None),    # one-CTA step 0, then the dense single pass
+                                      ((300, 1024), None),  # two-pass step 0, then the dense single pass
+                                      ((200, 512), 584)])   # strided rows: the row-wise kernels
+def test_delayed_nonfinite_step_records_nothing(bad_step, bad, shape, ld):
+    """A delayed step whose input holds a NaN/Inf sets FP8_ERR_NONFINITE and leaves the
+    history as it was; every later finite step is bit-exact with the oracle, which also
+    refuses the bad step and records nothing ([FFS] "数值验证看什么": non-finite values
+    are monitored, they must not reach the scale of the steps after them)."""
+    rows, cols = shape
+    h = 4
+    hist = fp8.History(h)
+    ring = np.zeros(h, np.float32)
+    ws = fp8.workspace_for(0, rows, 0, cols, fp8.FP8_SCALE_DELAYED)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for t in range(9):
+        x = mixed_input(rows, cols, seed=100 + t)
+        if t == bad_step:
+            x[rows // 2, cols // 3] = bad
+        st.zero_()
+        ring_before = hist.ring.cpu().numpy().copy()
+        q, s, d = fp8.empty_quant_outputs(rows, cols, fp8.FP8_SCALE_DELAYED, dequant=True)
+        fp8.fp8_quantize(_dev_rows(x, ld), fp8.FP8_E4M3, fp8.FP8_SCALE_DELAYED, q, s, hist=hist, dequant=d,
+                         dev_status=st, workspace=ws)
+        torch.cuda.synchronize()
+        assert hist.step == t + 1
+        assert hist.pending.item() == 0.0 and hist.ticket.item() == 0
+        if t == bad_step:
+            assert int(st.item()) == fp8.FP8_ERR_NONFINITE
+            with pytest.raises(oracle.OracleError):
+                oracle.delayed_step(x, fp8.FP8_E4M3, ring, t)
+            assert np.array_equal(hist.ring.cpu().numpy().view(np.uint32), ring_before.view(np.uint32)), \
+                "a non-finite step changed the history"
+            assert np.array_equal(ring.view(np.uint32), ring_before.view(np.uint32))
+            continue
+        assert int(st.item()) == 0, f"step {t}"
+        rq, rs, rd, _ = oracle.delayed_step(x, fp8.FP8_E4M3, ring, t, dequant=True)
+        assert s.cpu().numpy().view(np.uint32)[0] == np.float32(rs).view(np.uint32), f"step {t} scale"
+        assert first_mismatch(q.cpu().numpy(), rq) is None, f"step {t} codes"
+        assert first_mismatch(to_host_u16(d), rd) is None, f"step {t} dequant"
+        assert np.array_equal(hist.ring.cpu().numpy().view(np.uint32), ring.view(np.uint32)), f"step {t} ring"
+
+
+def test_quantize_nonfinite_sets_status_delayed():
+    """FP8_ERR_NONFINITE from the delayed mode at step 0 and at a later step."""
+    for cols in (256, 2048):
+        hist = fp8.History(16)
+        for t in range(3):
+            x = mixed_input(32, cols, seed=3 + t)
+            x[5, 17] = 0x7F80 if t != 1 else 0xFFC1
+            st = torch.zeros(1, dtype=torch.int32, device="cuda")
+            q, s, d = fp8.empty_quant_outputs(32, cols, fp8.FP8_SCALE_DELAYED)
+            fp8.fp8_quantize(to_dev_bf16(x), fp8.FP8_E4M3, fp8.FP8_SCALE_DELAYED, q, s, hist=hist, dev_status=st,
+                             workspace=fp8.workspace_for(0, 32, 0, cols, fp8.FP8_SCALE_DELAYED))
+            torch.cuda.synchronize()
+            assert int(st.item()) == fp8.FP8_ERR_NONFINITE, (cols, t)
+        assert np.all(hist.ring.cpu().numpy() == 0.0), "non-finite steps must record nothing"
+
+
+# ---------------------------------------------------------------- MX32 extreme groups
+def _mx_extreme_input(rows, cols, seed):
+    """32-element groups whose amax spans the whole bf16 range: groups made only of bf16
+    subnormals, normal groups below 2^-119 (the e = -127 clamp), groups just above it,
+    and groups up to the largest finite bf16; elements are every magnitude at or below
+    the group's amax (bf16 subnormals included), random signs."""
+    g = np.random.default_rng(seed)
+    ng = cols // 32
+    amax = g.integers(0x0001, 0x7F80, (rows, ng)).astype(np.uint32)
+    forced = np.array([0x0001, 0x0003, 0x003F, 0x0040, 0x007F, 0x0080, 0x0340, 0x0380, 0x03FF, 0x0400,
+                       0x0480, 0x7F7F, 0x0000], np.uint32)
+    amax[:, :min(ng, forced.size)] = forced[:min(ng, forced.size)]
+    mags = (g.random((rows, ng, 32)) * (amax[:, :, None] + 1)).astype(np.uint32)
+    # half of the elements at or below 2^-7 of the amax pattern's exponent: many subnormals
+    small = g.random((rows, ng, 32)) < 0.5
+    mags = np.where(small, mags & 0x00FF, mags)
+    mags = np.minimum(mags, amax[:, :, None])
+    pos = g.integers(0, 32, (rows, ng))
+    np.put_along_axis(mags, pos[:, :, None], amax[:, :, None], axis=2)
+    sign = g.integers(0, 2, (rows, ng, 32)).astype(np.uint32) << 15
+    return (mags | sign).astype(np.uint16).reshape(rows, cols)
+
+
+@pytest.mark.parametrize("shape,ld", [((64, 1024), None), ((130, 416), None), ((33, 2048), 2080),
+                                      ((3, 40960), None)])
+def test_mx_subnormal_and_clamped_groups(shape, ld):
+    """MX32 groups at the bottom of the bf16 range: the subnormal-amax branch of the
+    exponent and the clamp at e = -127 (byte 0x00), codes = encode(clip(x * 2^127));
+    scale bytes, codes and dequant bit-exact with the oracle."""
+    x = _mx_extreme_input(*shape, seed=shape[0] + shape[1])
+    check_parity(x, fp8.FP8_E4M3, fp8.FP8_SCALE_MX32, dequant=True, ld=ld, what=f"mx extremes {shape}")
+    _, e8, _ = oracle.quantize(x, oracle.E4M3, oracle.MX32, dequant=False)
+    assert (e8 == 0).sum() > 0 and ((e8 > 0) & (e8 < 20)).sum() > 0
+
+
+# ---------------------------------------------------------------- exhaustive cast sweep
+_FINITE_MAGS = np.arange(0, 0x7F80, dtype=np.uint32)                     # every finite |bf16| pattern
+_ALL_FINITE = np.concatenate([_FINITE_MAGS, _FINITE_MAGS | 0x8000]).astype(np.uint16)
+
+
+def _sweep_amax_patterns():
+    """>= 2,000 amax values: every 448 * 2^k and 57344 * 2^k that bf16 holds (power-of-two
+    scales s = 2^j in both formats, since 57344 / 448 = 128, so x / s is exact and lands
+    on every rounding midpoint of the FP8 grid, subnormal FP8 codes included), amax
+    values whose scale is the 1e-12 floor, and random bf16 patterns."""
+    pats = set()
+    for base in (448.0, 57344.0):
+        for k in range(-160, 130):
+            v = np.ldexp(np.float64(base), k)
+            if not (2.0 ** -133 <= v < 2.0 ** 128):
+                continue
+            b = int(inputs.bf16_bits(np.array([v], np.float32))[0])
+            if 0 < b < 0x7F80 and float(inputs.bf16_to_f32(np.array([b], np.uint16))[0]) == v:
+                pats.add(b)
+    pats.update([0x0001, 0x0100, 0x2000, 0x2B8C, 0x7F7F])   # near the 1e-12 floor; the largest finite bf16
+    g = np.random.default_rng(2024)
+    pats.update(int(v) for v in g.integers(1, 0x7F80, 1900))
+    return np.array(sorted(pats), np.uint32)
+
+
+def _exhaustive_rows(amax_pats, cols=16384):
+    """ROW sweep: for every amax A, rows holding A and every finite bf16 pattern (both
+    signs) with |x| <= A, 16,383 per row (the last row of A padded by repetition)."""
+    rows = []
+    for a in amax_pats:
+        p = _ALL_FINITE[(_ALL_FINITE & 0x7FFF) <= a]
+        per = cols - 1
+        nrow = -(-p.size // per)
+        p = np.resize(p, nrow * per).reshape(nrow, per)
+        rows.append(np.concatenate([p, np.full((nrow, 1), a, np.uint16)], axis=1))
+    return np.concatenate(rows, axis=0)
+
+
+def _exhaustive_blocks(amax_pats, cols=16384):
+    """1x128 sweep: blocks of 127 patterns (every finite pattern with |x| <= A, both signs)
+    plus A itself, for every amax A; blocks laid out 128 to a row."""
+    blocks = []
+    for a in amax_pats:
+        p = _ALL_FINITE[(_ALL_FINITE & 0x7FFF) <= a]
+        nb = -(-p.size // 127)
+        p = np.resize(p, nb * 127).reshape(nb, 127)
+        blocks.append(np.concatenate([np.full((nb, 1), a, np.uint16), p], axis=1))
+    b = np.concatenate(blocks, axis=0)
+    per_row = cols // 128
+    nrow = -(-b.shape[0] // per_row)
+    b = np.resize(b, (nrow * per_row, 128))
+    return b.reshape(nrow, cols)
+
+
+@pytest.mark.parametrize("mode", [fp8.FP8_SCALE_ROW, fp8.FP8_SCALE_BLOCK_1x128])
+def test_cast_exhaustive_every_finite_bf16_pattern(mode):
+    """Every finite bf16 pattern, both signs, through the cast under each of >= 2,000
+    scales (one per row, or one per 1x128 block) and both formats, codes and dequant
+    bit-exact with the oracle.  The power-of-two scales put x / s exactly on the FP8
+    rounding midpoints (ties), where the kernel's reciprocal-plus-correction division
+    must still equal the IEEE quotient ([FFS] "Scale 怎样把 Tensor 塞进 E4M3":
+    X_fp8 = cast(clip(X / s)))."""
+    amax = _sweep_amax_patterns()
+    assert amax.size >= 2000
+    x = _exhaustive_rows(amax) if mode == fp8.FP8_SCALE_ROW else _exhaustive_blocks(amax)
+    for fmt in FMTS:
+        check_parity(x, fmt, mode, dequant=True, what=f"exhaustive mode {mode} fmt {fmt}")

@@ -301,7 +301,82 @@ def test_mx32_exponent_range_and_codes():
     assert oracle.mx_exponent(0.0) == -127
 
 
+def _frexp_floor_log2(v: float) -> int:
+    """floor(log2 v) of a positive float through Python's own frexp (independent of the oracle)."""
+    import math
+    return math.frexp(v)[1] - 1
+
+
+def test_mx32_subnormal_and_clamped_groups():
+    """Groups whose amax is a bf16 subnormal, or a normal below 2^-119, reach the lower
+    clamp e = -127 ([FFS] "Per-channel 与 Block Scaling": one power-of-two scale per 32
+    values; e = clamp(floor(log2 amax) - 8, -127, 127)): the scale byte is 0x00 and the
+    codes are the nearest-code encoding of clip(x * 2^127), which the NumPy brute-force
+    encoder computes here independently.  Groups just above the clamp keep e exact."""
+    from oracle import numpy_encoder
+    # amax patterns: bf16 subnormals 2^-133, 3*2^-132, 2^-127 (0x0040), and normals
+    # 1.5*2^-121, 2^-120, 2^-119 (e = -127 exactly), 2^-118 (e = -126), 1.75*2^-101
+    amax_bits = np.array([0x0001, 0x0003, 0x0040, 0x0340, 0x0380, 0x0400, 0x0480, 0x0D60], np.uint16)
+    g = np.random.default_rng(23)
+    x = np.zeros((4, 32 * amax_bits.size), np.uint16)
+    for j, a in enumerate(amax_bits):
+        # every element of the group at or below its amax pattern, random signs; the
+        # amax itself at a random position
+        mags = g.integers(0, int(a) + 1, (4, 32)).astype(np.uint16)
+        mags[np.arange(4), g.integers(0, 32, 4)] = a
+        sign = (g.integers(0, 2, (4, 32)) << 15).astype(np.uint16)
+        x[:, 32 * j:32 * (j + 1)] = mags | sign
+    q, e8, d = oracle.quantize(x, E4M3, oracle.MX32, dequant=True)
+    amax_f = inputs.bf16_to_f32(amax_bits).astype(np.float64)
+    e_expect = np.array([min(127, max(-127, _frexp_floor_log2(v) - 8)) for v in amax_f])
+    assert e_expect[:6].tolist() == [-127] * 6 and e_expect[6] == -126 and e_expect[7] == -109
+    assert np.array_equal(e8.astype(np.int64) - 127, np.tile(e_expect, (4, 1)))
+    assert np.all(e8[:, :6] == 0)
+    xf = inputs.bf16_to_f32(x).astype(np.float64)
+    t = np.clip(xf * np.exp2(-np.repeat(e_expect, 32))[None, :], -448.0, 448.0)
+    ref = numpy_encoder.encode_nearest(t.ravel(), E4M3).reshape(q.shape)
+    assert np.array_equal(q, ref)
+    # dequant: decode(q) * 2^e, exact in fp32, then bf16 (here every value is a bf16 value
+    # or a bf16 subnormal rounding case handled by the torch cast)
+    import torch
+    table = numpy_encoder.value_table(E4M3)
+    dq = (table[q] * np.exp2(np.repeat(e_expect, 32))[None, :]).astype(np.float32)
+    dt = torch.from_numpy(dq).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(d, dt)
+
+
 # ------------------------------------------------------------ delayed scaling
+def test_delayed_nonfinite_step_records_nothing():
+    """A step whose input holds a NaN or an Inf is refused and leaves the history as it
+    was; the steps after it take their scale from the window of the valid steps only
+    (written out here as a plain list of the amax of each valid step)."""
+    g = np.random.default_rng(29)
+    h = 4
+    ring = np.zeros(h, np.float32)
+    slot_amax = {}                      # slot -> amax of the last valid step that wrote it
+    for t in range(11):
+        x = inputs.bf16_bits((g.standard_normal((8, 64)) * (1 + t)).astype(np.float32))
+        if t in (2, 7):
+            x[3, 5] = 0x7F80 if t == 2 else 0xFFC1        # +Inf, NaN
+            before = ring.copy()
+            with pytest.raises(oracle.OracleError):
+                oracle.delayed_step(x, E4M3, ring, t)
+            assert np.array_equal(ring.view(np.uint32), before.view(np.uint32))
+            continue
+        xf = inputs.bf16_to_f32(x)
+        amax_t = np.float32(np.abs(xf).max())
+        q, s, _, _ = oracle.delayed_step(x, E4M3, ring, t)
+        if t == 0:
+            hist = amax_t
+        else:
+            hist = np.float32(max(slot_amax.values(), default=np.float32(0)))
+        assert s == np.float32(max(hist, np.float32(1e-12)) / np.float32(448.0)), t
+        assert np.array_equal(q, oracle.quant_scaled(xf.ravel(), s, E4M3).reshape(q.shape))
+        slot_amax[t % h] = amax_t
+    # slot 2 % 4 = 2 was last written by step 10; slot 7 % 4 = 3 by step 3 (step 7 was refused)
+    assert ring[3] == slot_amax[3]
+
+
 def test_delayed_ring_semantics():
     g = np.random.default_rng(19)
     h = 4
@@ -414,3 +489,61 @@ def test_tolerance_rule_rejects_planted_error():
     ok, _, _ = oracle.gemm_within_tolerance(bad, y, bound)
     assert not ok.any()
     assert oracle.bf16_ulp(np.array([1.0]))[0] == 2 ** -7
+
+
+def test_results_do_not_depend_on_the_thread_count():
+    """The oracle splits rows (and output points) over threads; every mode gives the same
+    bits on 1 thread and on several, including the ragged last range."""
+    x = inputs.bf16_bits((np.random.default_rng(31).standard_normal((259, 512))
+                          * np.exp(np.random.default_rng(32).standard_normal((259, 1)))).astype(np.float32))
+    w = inputs.bf16_bits((np.random.default_rng(33).standard_normal((140, 512)) * 0.02).astype(np.float32))
+    prev = oracle.get_threads()
+    try:
+        outs = {}
+        for n in (1, 5):
+            oracle.set_threads(n)
+            res = [oracle.quantize(x, fmt, mode) for fmt in (E4M3, E5M2) for mode in
+                   (oracle.TENSOR, oracle.ROW, oracle.BLOCK_1x128, oracle.BLOCK_128x128)]
+            res.append(oracle.quantize(x, E4M3, oracle.MX32))
+            ring = np.zeros(4, np.float32)
+            res.append(tuple(oracle.delayed_step(x, E4M3, ring, t)[:2] for t in range(3)) + (ring.copy(),))
+            qa, sa, _ = oracle.quantize(x, E4M3, oracle.ROW, dequant=False)
+            qb, sb, _ = oracle.quantize(w, E4M3, oracle.ROW, dequant=False)
+            pm = np.repeat(np.arange(259), 7)
+            pn = np.tile(np.arange(0, 140, 20), 259)
+            res.append(oracle.gemm_ref_points(qa, sa, oracle.ROW, E4M3, qb, sb, oracle.ROW, E4M3, pm, pn))
+            outs[n] = res
+        def flat(r):
+            out = []
+            for v in r:
+                if isinstance(v, (tuple, list)):
+                    out.extend(flat(v))
+                elif v is not None:
+                    out.append(np.atleast_1d(np.asarray(v)))
+            return out
+        a, b = flat(outs[1]), flat(outs[5])
+        assert len(a) == len(b)
+        for u, v in zip(a, b):
+            assert np.array_equal(u.view(np.uint8) if u.dtype.kind == "f" else u,
+                                  v.view(np.uint8) if v.dtype.kind == "f" else v)
+    finally:
+        oracle.set_threads(prev)
+
+
+def test_gemm_ref_rows_agrees_with_the_pointwise_reference():
+    """gemm_ref_rows (fp64 BLAS over exactly dequantised operands) against the C
+    reference at every output of small problems in every scale mode, to fp64 rounding."""
+    g = np.random.default_rng(37)
+    cases = [(oracle.ROW, oracle.ROW, E4M3, E5M2), (oracle.TENSOR, oracle.TENSOR, E5M2, E5M2),
+             (oracle.BLOCK_1x128, oracle.BLOCK_128x128, E4M3, E4M3), (oracle.MX32, oracle.MX32, E4M3, E4M3)]
+    for am, bm, fa, fb in cases:
+        M, N, K = 130, 260, 384
+        x = inputs.bf16_bits((g.standard_normal((M, K)) * np.exp(g.standard_normal((M, 1)))).astype(np.float32))
+        w = inputs.bf16_bits((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+        qa, sa, _ = oracle.quantize(x, fa, am, dequant=False)
+        qb, sb, _ = oracle.quantize(w, fb, bm, dequant=False)
+        y, bnd = oracle.gemm_ref_full(qa, sa, am, fa, qb, sb, bm, fb)
+        rows = np.array([0, 1, 64, 127, 128, 129])
+        y2, b2 = oracle.gemm_ref_rows(qa, sa, am, fa, qb, sb, bm, fb, rows, chunk=100)
+        assert np.allclose(y2, y[rows], rtol=0, atol=1e-12 * bnd[rows].max())
+        assert np.allclose(b2, bnd[rows], rtol=1e-12, atol=0)
