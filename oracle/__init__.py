@@ -64,6 +64,8 @@ def _load():
                                         P, P, I64, P, P]
     lib.orc_gemm_ref_full.restype = I32
     lib.orc_gemm_ref_full.argtypes = [P, P, I32, I32, P, P, I32, I32, I64, I64, I64, P, P]
+    lib.orc_gemm_ref_slice.restype = I32
+    lib.orc_gemm_ref_slice.argtypes = [P, P, I32, I32, P, P, I32, I32, I64, I64, I64, I64, I64, P, P]
     lib.orc_decode_table.restype, lib.orc_decode_table.argtypes = None, [I32, P]
     for name in ("orc_encode_array", "orc_encode_bruteforce_array"):
         getattr(lib, name).restype = None
@@ -268,6 +270,21 @@ def gemm_ref_full(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b):
                                    _ptr(y), _ptr(bound))
     if rc != 0:
         raise OracleError("orc_gemm_ref_full failed")
+    return y, bound
+
+
+def gemm_ref_slice(a, sa, a_mode, fmt_a, b, sb, b_mode, fmt_b, m0: int, m1: int):
+    """fp64 reference of the output rows m0..m1-1 against every row of B (the C oracle,
+    rows of B split over the threads); returns (y, bound), each [m1 - m0, N]."""
+    M, K = a.shape
+    N = b.shape[0]
+    y = np.empty((m1 - m0, N), np.float64)
+    bound = np.empty((m1 - m0, N), np.float64)
+    rc = _load().orc_gemm_ref_slice(_ptr(np.ascontiguousarray(a)), _ptr(np.ascontiguousarray(sa)), a_mode, fmt_a,
+                                    _ptr(np.ascontiguousarray(b)), _ptr(np.ascontiguousarray(sb)), b_mode, fmt_b,
+                                    M, N, K, m0, m1, _ptr(y), _ptr(bound))
+    if rc != 0:
+        raise OracleError("orc_gemm_ref_slice failed")
     return y, bound
 
 

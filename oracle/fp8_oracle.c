@@ -661,6 +661,61 @@ int orc_gemm_ref_full(const uint8_t* a, const void* sa, int a_mode, int fmt_a,
     return 0;
 }
 
+/* Whole output rows [m0, m1) x all N (y and bound are [m1 - m0, N]): the operand rows
+ * of A are dequantised once; the N rows of B are split over the threads, each
+ * dequantising one row of B at a time (memory stays at K doubles per thread). */
+typedef struct {
+    const uint8_t* b;
+    const void* sb;
+    int b_mode, fmt_b;
+    const double* da;
+    int64_t rows, N, K;
+    double *y, *bound;
+    int err_part[ORC_MAX_THREADS];
+} rjob;
+
+static void rows_range(void* c, int64_t n0, int64_t n1, int part) {
+    rjob* j = (rjob*)c;
+    double* rb = (double*)malloc(sizeof(double) * (size_t)(j->K > 0 ? j->K : 1));
+    j->err_part[part] = rb == NULL;
+    if (!rb) return;
+    for (int64_t n = n0; n < n1; ++n) {
+        deq_row(j->b, j->sb, j->b_mode, j->fmt_b, n, j->K, rb);
+        for (int64_t i = 0; i < j->rows; ++i) {
+            const double* ra = j->da + i * j->K;
+            double acc = 0.0, bnd = 0.0;
+            for (int64_t k = 0; k < j->K; ++k) {
+                double p = ra[k] * rb[k];
+                acc += p;
+                bnd += fabs(p);
+            }
+            j->y[i * j->N + n] = acc;
+            j->bound[i * j->N + n] = bnd;
+        }
+    }
+    free(rb);
+}
+
+int orc_gemm_ref_slice(const uint8_t* a, const void* sa, int a_mode, int fmt_a,
+                      const uint8_t* b, const void* sb, int b_mode, int fmt_b,
+                      int64_t M, int64_t N, int64_t K, int64_t m0, int64_t m1,
+                      double* y, double* bound) {
+    if (m0 < 0 || m1 > M || m0 > m1) return 2;
+    rjob* j = (rjob*)calloc(1, sizeof(rjob));
+    double* da = (double*)malloc(sizeof(double) * (size_t)((m1 - m0) * K > 0 ? (m1 - m0) * K : 1));
+    if (!j || !da) { free(j); free(da); return 2; }
+    for (int64_t m = m0; m < m1; ++m) deq_row(a, sa, a_mode, fmt_a, m, K, da + (m - m0) * K);
+    j->b = b; j->sb = sb; j->b_mode = b_mode; j->fmt_b = fmt_b; j->da = da;
+    j->rows = m1 - m0; j->N = N; j->K = K; j->y = y; j->bound = bound;
+    int parts = orc_parallel(N, 1, j, rows_range);
+    int rc = 0;
+    for (int k = 0; k < parts; ++k)
+        if (j->err_part[k]) rc = 2;
+    free(da);
+    free(j);
+    return rc;
+}
+
 /* Decoded values of every code of a format, for table-driven checks. */
 void orc_decode_table(int fmt, double* out256) {
     for (int c = 0; c < 256; ++c) out256[c] = orc_decode((uint8_t)c, fmt);
