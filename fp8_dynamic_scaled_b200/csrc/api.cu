@@ -43,7 +43,7 @@ int64_t scale_bytes(int32_t mode, int64_t rows, int64_t cols) {
     }
 }
 
-size_t partials_bytes() { return align_up(4 * (size_t)amax_partials_count(), 256); }
+size_t partials_bytes() { return align_up(kTensorWorkspaceBytes, 256); }
 
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA; }
 

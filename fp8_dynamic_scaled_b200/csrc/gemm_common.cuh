@@ -24,10 +24,6 @@ constexpr uint32_t B_STAGE_BYTES = BN * BK;   // 32 KB
 constexpr uint64_t WAIT_TIMEOUT_NS = 4000000000ull;   // 4 s: default limit of a pipeline wait
 constexpr uint64_t DRAIN_LIMIT_NS = 2000000000ull;    // 2 s: limit of a wait for hardware completion
 
-// Limit of the pipeline waits of the kernels launched next from this process (0: the
-// default WAIT_TIMEOUT_NS).  Set only through the testing entry point that exercises
-// the failure path (fp8_testing_set_wait_limit_ns); read when a launch is prepared.
-uint64_t wait_limit_ns();
 
 struct GemmParams {
     int32_t M, N, K;
@@ -73,6 +69,19 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
                                              int32_t* status, uint64_t limit_ns) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer();
+    if (limit_ns < 1000000ull) {
+        // a short limit (the failure-path tests): each test suspends the thread for at most
+        // 100 ns, so that the limit is checked well before a slow phase could complete
+        while (true) {
+            if (ptx::mbar_try_wait_hint(bar, parity, 100u)) return true;
+            if (*abort_flag) return false;
+            if (ptx::globaltimer() - t0 > limit_ns) {
+                *abort_flag = 1;
+                report_status(status, FP8_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
@@ -329,7 +338,32 @@ __device__ __forceinline__ void rowscale_chunk(const GemmParams& p, EpiState& es
     }
 }
 
+// Tile raster: the operand with the smaller footprint is walked fastest, in groups
+// of `group` tiles whose panels fit comfortably in L2; within a group the fast index
+// varies fastest and the group sweeps the whole slow dimension before the next group.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int32_t t, int32_t& mb, int32_t& nb) {
+    const int32_t nfast = p.m_fastest ? p.num_m : p.num_n;
+    const int32_t nslow = p.m_fastest ? p.num_n : p.num_m;
+    const int32_t per_group = p.group * nslow;
+    const int32_t g = t / per_group;
+    const int32_t rem = t - g * per_group;
+    const int32_t width = min(p.group, nfast - g * p.group);
+    const int32_t fast = g * p.group + rem % width;
+    const int32_t slow = rem / width;
+    if (p.m_fastest) { mb = fast; nb = slow; }
+    else             { nb = fast; mb = slow; }
+}
+
 // ================================================================ host side
+// Raster group for a given row-tile height (see tile_coords).
+inline int32_t raster_group(int64_t nfast, int64_t panel_bytes) {
+    int64_t grp = std::max<int64_t>(1, (int64_t)36 * 1024 * 1024 / std::max<int64_t>(panel_bytes, 1));
+    if (grp >= nfast) return (int32_t)std::max<int64_t>(nfast, 1);
+    const int64_t ngroups = (nfast + grp - 1) / grp;
+    return (int32_t)std::max<int64_t>((nfast + ngroups - 1) / ngroups, 1);
+}
+
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);

@@ -72,22 +72,6 @@ struct Smem {
     static constexpr uint32_t ALLOC = TOTAL + 1024;             // slack for 1024-B alignment
 };
 
-// Tile raster: the operand with the smaller footprint is walked fastest, in groups
-// of `group` tiles whose panels fit comfortably in L2; within a group the fast index
-// varies fastest and the group sweeps the whole slow dimension before the next group.
-__device__ __forceinline__ void tile_coords(const GemmParams& p, int32_t t, int32_t& mb, int32_t& nb) {
-    const int32_t nfast = p.m_fastest ? p.num_m : p.num_n;
-    const int32_t nslow = p.m_fastest ? p.num_n : p.num_m;
-    const int32_t per_group = p.group * nslow;
-    const int32_t g = t / per_group;
-    const int32_t rem = t - g * per_group;
-    const int32_t width = min(p.group, nfast - g * p.group);
-    const int32_t fast = g * p.group + rem % width;
-    const int32_t slow = rem / width;
-    if (p.m_fastest) { mb = fast; nb = slow; }
-    else             { nb = fast; mb = slow; }
-}
-
 // ================================================================ the kernel
 template <int V, bool EXT>
 __global__ void __launch_bounds__(Smem<V>::NT, 1)
@@ -759,14 +743,6 @@ static cudaError_t launch_variant(const GemmArgs& g, const GemmParams& p, cudaSt
     cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<V, EXT>, ta, tb, ty, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
-}
-
-// Raster group for a given row-tile height (see tile_coords).
-static int32_t raster_group(int64_t nfast, int64_t panel_bytes) {
-    int64_t grp = std::max<int64_t>(1, (int64_t)36 * 1024 * 1024 / std::max<int64_t>(panel_bytes, 1));
-    if (grp >= nfast) return (int32_t)std::max<int64_t>(nfast, 1);
-    const int64_t ngroups = (nfast + grp - 1) / grp;
-    return (int32_t)std::max<int64_t>((nfast + ngroups - 1) / ngroups, 1);
 }
 
 // CTA-pair launch: clusters of two CTAs, 256 x 256 tiles.

@@ -29,6 +29,13 @@ struct QuantArgs {
 };
 
 int32_t amax_partials_count();
+// The per-tensor workspace (fp8_workspace_size for TENSOR / DELAYED): the u32 partial
+// maxima of the two-pass kernels, then the single-launch kernel's call counter and
+// its per-CTA slots (8-byte words).
+constexpr size_t kPartialsBytes = 4864;              // 4 * 1184 rounded up to 256
+constexpr size_t kEpochOffset = kPartialsBytes;
+constexpr size_t kSlotsOffset = kEpochOffset + 256;
+constexpr size_t kTensorWorkspaceBytes = kSlotsOffset + 8 * 1184;
 cudaError_t launch_quantize_tensor(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_quantize_grouped(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_fill_scale(float* s, int64_t n, float v, cudaStream_t st);
@@ -60,9 +67,12 @@ struct GemmArgs {
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
 
-// Limit of every pipeline wait in the kernels launched from now on (0: the default);
-// only the testing entry point fp8_testing_set_wait_limit_ns calls this.
+// Limit of every pipeline wait (and of the per-tensor kernel's grid-wide exchange) in
+// the kernels launched from now on (0: the default, 4 s); only the testing entry point
+// fp8_testing_set_wait_limit_ns sets it.  wait_limit_ns() is read when a launch is
+// prepared.
 void set_wait_limit_ns(uint64_t ns);
+uint64_t wait_limit_ns();
 
 struct WoArgs {              // weight-only FP8 linear (wo_sm100.cu)
     const uint16_t* x;       // bf16 [M, K], row stride ldx

@@ -16,6 +16,7 @@
 // patterns (exact and order-free); a pattern >= 0x7F80 flags NaN/Inf input.
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace fp8b {
 
@@ -778,6 +779,227 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const
     }
 }
 
+// ================================================================ per-tensor in one launch
+// Current per-tensor scaling needs the whole tensor's a_max before the first code can be
+// written ([FFS] "Current Scaling": the amax sits on the critical path).  The two-pass
+// kernels above read X twice.  This kernel runs one CTA per SM, all resident at once (a
+// cooperative launch), in two phases around one grid-wide exchange of the amax:
+//   own   each CTA owns one contiguous piece of X at the front of the tensor: the first
+//         PT_HELD_BYTES of it are bulk-copied into shared memory, the rest (up to
+//         PT_THREADS * PT_REG_VEC vectors) loaded into registers; both stay on chip
+//         across the exchange;
+//   spill the rest of X, in chunks of PT_SLOT_BYTES dealt round-robin to the CTAs
+//         (chunk c to CTA c mod G, so every CTA's share is spread over the whole tensor),
+//         streamed through a ring of shared-memory slots filled by bulk copies (many
+//         bytes in flight, no registers): for its amax in phase 1, and again, from the
+//         last chunk back (the ones the L2 cache still holds), for the cast in phase 2.
+// The exchange: every CTA writes its amax into its own slot of the workspace, tagged
+// with this call's number, and reads all the slots back (a bounded wait).  The codes
+// are those of rq_amax + rq_tensor<CAST> bit for bit: the same integer max over |bf16|
+// patterns and the same cast.
+//
+// The call number: the workspace keeps a 32-bit counter E.  Every CTA reads E before it
+// writes its slot, and CTA 0 stores E + 1 only after it has seen every slot, i.e. after
+// every CTA has read E; the slots of call E + 1 carry the tag E + 1, so the slots of an
+// earlier call (tag <= E) are never taken for this one, whatever the workspace held
+// before (a stale or uninitialised slot would also have to match a 16-bit check of its
+// tag and CTA).  CUDA-graph replays advance E the same way.
+constexpr int PT_THREADS = 512;
+constexpr int PT_REG_VEC = 16;                      // 16-byte vectors per thread kept in registers
+constexpr uint32_t PT_HELD_BYTES = 96 * 1024;       // bytes per CTA kept in shared memory
+constexpr int PT_HELD_CHUNKS = 6;                   // its bulk copies (one mbarrier each)
+constexpr int PT_RING = 4;                          // spill ring slots
+constexpr uint32_t PT_SLOT_BYTES = 24 * 1024;       // bytes per slot: 3 vectors per thread
+constexpr int64_t PT_SLOT_VEC = PT_SLOT_BYTES / 16;
+constexpr int64_t PT_OWN_VEC = PT_HELD_BYTES / 16 + (int64_t)PT_THREADS * PT_REG_VEC;
+constexpr uint32_t PT_DYN_SMEM = PT_HELD_BYTES + PT_RING * PT_SLOT_BYTES + 8 * (PT_HELD_CHUNKS + PT_RING);
+constexpr int64_t PT_MIN_ELEMS = (int64_t)16 << 20; // smaller tensors: the two-pass kernels (L2 holds X)
+
+struct PTParams {
+    const uint16_t* x;
+    int64_t nvec;                  // 16-byte vectors in X
+    uint8_t* q;
+    float* scale;
+    uint16_t* deq;
+    int32_t* status;
+    uint32_t* epoch;               // workspace: the call counter E
+    unsigned long long* slots;     // workspace: one tagged amax per CTA
+    float* ring;                   // delayed scaling, step 0: ring[slot] = amax (nullable)
+    int32_t slot;
+    uint64_t wait_ns;              // limit of the exchange wait
+};
+
+__device__ __forceinline__ uint32_t pt_check(uint32_t tag, uint32_t cta) {
+    return ((tag * 0x9E3779B1u) ^ (cta * 0x85EBCA77u) ^ 0xA5A5u) >> 16;
+}
+
+// A wait for bulk copies this CTA issued (hardware completion; bounded, not cut short).
+__device__ __forceinline__ bool pt_wait_copy(uint64_t* bar, uint32_t parity, int32_t* status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer() - t0 > 2000000000ull) {
+            report_status(status, FP8_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <int FMT, bool DEQ>
+__global__ void __launch_bounds__(PT_THREADS, 1) rq_persist_kernel(const PTParams p) {
+    extern __shared__ __align__(1024) uint8_t pt_smem[];
+    uint8_t* held = pt_smem;
+    uint8_t* ring = pt_smem + PT_HELD_BYTES;
+    uint64_t* hbar = reinterpret_cast<uint64_t*>(pt_smem + PT_HELD_BYTES + PT_RING * PT_SLOT_BYTES);
+    uint64_t* rbar = hbar + PT_HELD_CHUNKS;
+    __shared__ uint32_t red[32];
+    __shared__ uint32_t s_epoch;
+    const int t = threadIdx.x;
+    const int64_t G = gridDim.x, b = blockIdx.x;
+    // this CTA's own piece [v0, v1): held part [v0, r0), registers [r0, v1)
+    const int64_t v0 = min(p.nvec, b * PT_OWN_VEC), v1 = min(p.nvec, v0 + PT_OWN_VEC);
+    const int64_t n_held = min(v1 - v0, (int64_t)(PT_HELD_BYTES / 16));
+    const int64_t r0 = v0 + n_held;
+    // the spill: everything past the own pieces, in chunks of PT_SLOT_VEC vectors
+    const int64_t sp0 = min(p.nvec, G * PT_OWN_VEC);
+    const int64_t nsc = (p.nvec - sp0 + PT_SLOT_VEC - 1) / PT_SLOT_VEC;
+    const uint4* xv = reinterpret_cast<const uint4*>(p.x);
+    const uint32_t held_bytes = (uint32_t)(n_held * 16);
+    const uint32_t hchunk = (held_bytes / PT_HELD_CHUNKS + 15u) & ~15u;   // a multiple of 16
+    const int nhc = hchunk ? (int)((held_bytes + hchunk - 1) / hchunk) : 0;
+    // this CTA's spill chunks: c = b + i G in phase 1 (i < nb), then c = nsc - 1 - b - i G
+    // in phase 2; ring use j < 2 nb goes to slot j % PT_RING with parity (j / PT_RING) & 1
+    const int64_t nb = b < nsc ? (nsc - 1 - b) / G + 1 : 0;
+    auto chunk_of = [&](int64_t j) { return j < nb ? b + j * G : (nsc - 1 - b) - (j - nb) * G; };
+
+    if (t == 0) {
+        s_epoch = *reinterpret_cast<volatile uint32_t*>(p.epoch);   // read before this CTA arrives
+        for (int c = 0; c < PT_HELD_CHUNKS + PT_RING; ++c) ptx::mbar_init(&hbar[c], 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();                                   // the barriers and s_epoch are set
+    const uint32_t tag = s_epoch + 1u;
+    const uint64_t pol_keep = ptx::createpolicy_evict_last(), pol_drop = ptx::createpolicy_evict_first();
+    // one thread: copy the chunk of ring use j into its slot (the first read keeps its
+    // lines in L2 for the re-read; the re-read drops them)
+    auto issue = [&](int64_t j) {
+        const int64_t cv0 = sp0 + chunk_of(j) * PT_SLOT_VEC;
+        const uint32_t bytes = (uint32_t)(min(PT_SLOT_VEC, p.nvec - cv0) * 16);
+        const int sl = (int)(j % PT_RING);
+        ptx::mbar_arrive_expect_tx(&rbar[sl], bytes);
+        ptx::bulk_load_1d_hint(ring + sl * PT_SLOT_BYTES, xv + cv0, bytes, &rbar[sl], j < nb ? pol_keep : pol_drop);
+    };
+    // ring uses [j0, j1): fn(slot vectors, first vector index of the chunk, count); the
+    // copy of use j + PT_RING (up to jmax) goes out as soon as slot j is free
+    auto run_ring = [&](int64_t j0, int64_t j1, int64_t jmax, auto&& fn) -> bool {
+        bool ok = true;
+        for (int64_t j = j0; j < j1; ++j) {
+            const int sl = (int)(j % PT_RING);
+            ok &= pt_wait_copy(&rbar[sl], (uint32_t)((j / PT_RING) & 1), p.status);
+            const int64_t cv0 = sp0 + chunk_of(j) * PT_SLOT_VEC;
+            fn(reinterpret_cast<const uint4*>(ring + sl * PT_SLOT_BYTES), cv0, min(PT_SLOT_VEC, p.nvec - cv0));
+            __syncthreads();                           // every thread is done with slot sl
+            if (t == 0 && j + PT_RING < jmax) issue(j + PT_RING);
+        }
+        return ok;
+    };
+    if (t == 0) {
+        for (int c = 0; c < nhc; ++c) {
+            const uint32_t off = (uint32_t)c * hchunk;
+            const uint32_t nbytes = min(hchunk, held_bytes - off);
+            ptx::mbar_arrive_expect_tx(&hbar[c], nbytes);
+            ptx::bulk_load_1d_hint(held + off, reinterpret_cast<const uint8_t*>(xv + v0) + off, nbytes, &hbar[c],
+                                   pol_drop);
+        }
+        for (int64_t j = 0; j < min(2 * nb, (int64_t)PT_RING); ++j) issue(j);
+    }
+    // ---- phase 1: a_max of the registers, the spill chunks and the held part
+    uint4 reg[PT_REG_VEC];
+#pragma unroll
+    for (int j = 0; j < PT_REG_VEC; ++j) {
+        const int64_t k = r0 + t + (int64_t)PT_THREADS * j;
+        reg[j] = k < v1 ? ld_v4_stream(xv + k) : make_uint4(0, 0, 0, 0);
+    }
+    uint32_t m2 = 0;
+    // phase 1's ring also sends out phase 2's first copies as the ring empties
+    bool fail = !run_ring(0, nb, 2 * nb, [&](const uint4* sv, int64_t, int64_t nv) {
+        for (int64_t k = t; k < nv; k += PT_THREADS) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(sv[k]));
+    });
+#pragma unroll
+    for (int j = 0; j < PT_REG_VEC; ++j) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(reg[j]));
+    for (int c = 0; c < nhc; ++c) fail |= !pt_wait_copy(&hbar[c], 0, p.status);
+    for (int64_t k = t; k < n_held; k += PT_THREADS)
+        m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(*reinterpret_cast<const uint4*>(held + k * 16)));
+    const uint32_t m_cta = block_max_u32(hmax_pair(m2 & 0x7FFF7FFFu), red);
+    // ---- the exchange
+    if (t == 0) {
+        const unsigned long long word = ((unsigned long long)tag << 32) |
+                                        ((unsigned long long)pt_check(tag, (uint32_t)b) << 16) | m_cta;
+        atomicExch(p.slots + b, word);
+    }
+    uint32_t gm = 0;
+    if (!fail) {
+        const uint64_t t0 = ptx::globaltimer();
+        for (int64_t i = t; i < G && !fail; i += PT_THREADS) {
+            const volatile unsigned long long* sp = p.slots + i;
+            while (true) {
+                const unsigned long long w = *sp;
+                if ((uint32_t)(w >> 32) == tag && (uint32_t)((w >> 16) & 0xFFFFu) == pt_check(tag, (uint32_t)i)) {
+                    gm = max(gm, (uint32_t)(w & 0xFFFFu));
+                    break;
+                }
+                if (ptx::globaltimer() - t0 > p.wait_ns) {
+                    report_status(p.status, FP8_ERR_TIMEOUT);
+                    fail = true;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+    }
+    fail = __syncthreads_or(fail) != 0;
+    // CTA 0 advances the call counter once its wait has ended, whether or not the exchange
+    // completed: on success every CTA has read E by then (it arrived).  (After a time-out a
+    // CTA that had not even started could still read the new value; the workspace is then
+    // undefined until the caller zeroes it, which the interface states.)
+    if (b == 0 && t == 0) *reinterpret_cast<volatile uint32_t*>(p.epoch) = tag;
+    if (fail) {
+        // outputs unspecified; phase 2's copies already issued must land before the CTA exits
+        if (t == 0)
+            for (int64_t j = nb; j < min(2 * nb, nb + (int64_t)PT_RING); ++j)
+                pt_wait_copy(&rbar[j % PT_RING], (uint32_t)((j / PT_RING) & 1), p.status);
+        return;
+    }
+    gm = block_max_u32(gm, red);
+    const bool finite_in = gm < 0x7F80u;
+    if (!finite_in) {
+        if (b == 0 && t == 0) report_status(p.status, FP8_ERR_NONFINITE);
+        gm = 0x7F7Fu;                                  // keep the scale finite; outputs unspecified
+    }
+    const RcpScale op = rcp_scale_from_amax_bits<FMT>(gm);
+    if (b == 0 && t == 0) {
+        p.scale[0] = op.s;
+        if (p.ring != nullptr && finite_in) p.ring[p.slot] = bf16bits_to_float(gm);
+    }
+    pdl_launch_dependents();                           // a dependent GEMM may start streaming its other operand
+    // ---- phase 2: the cast of the spill (from the last chunk back), registers, held part
+    auto emit = [&](int64_t k, const uint4& a) {
+        const uint2 cq = cast_vec_rcp<FMT>(a, op);
+        __stcs(reinterpret_cast<uint2*>(p.q) + k, cq);
+        if (DEQ) st_v4_stream(p.deq + k * VEC, dequant_vec2<FMT>(cq, op.s));
+    };
+    run_ring(nb, 2 * nb, 2 * nb, [&](const uint4* sv, int64_t cv0, int64_t nv) {
+        for (int64_t k = t; k < nv; k += PT_THREADS) emit(cv0 + k, sv[k]);
+    });
+#pragma unroll
+    for (int j = 0; j < PT_REG_VEC; ++j) {
+        const int64_t k = r0 + t + (int64_t)PT_THREADS * j;
+        if (k < v1) emit(k, reg[j]);
+    }
+    for (int64_t k = t; k < n_held; k += PT_THREADS) emit(v0 + k, *reinterpret_cast<const uint4*>(held + k * 16));
+}
+
 // ================================================================ launchers
 static int sm_count_cached() {
     static int cache[kDeviceCacheSlots];   // per device
@@ -822,6 +1044,51 @@ static void launch_cast_tensor(const QuantArgs& a, int src, dim3 grid, int npart
 
 static int64_t rq_grid_cap() { return std::min<int64_t>(amax_partials_count(), (int64_t)sm_count_cached() * 8); }
 
+// Cooperative launch of rq_persist_kernel (all CTAs resident at once), one grid per
+// SM count times the CTAs that fit per SM (known per device, at most one slot per CTA).
+// `launched` stays false when the kernel cannot run here (the caller then takes the
+// two-pass kernels).
+template <int FMT, bool DEQ>
+static cudaError_t launch_persist(const PTParams& pt, cudaStream_t st, bool& launched) {
+    static int ctas_per_sm[kDeviceCacheSlots];      // 0: unknown, -1: not usable, else CTAs per SM
+    const int ds = device_slot();
+    int per_sm = ds >= 0 ? ctas_per_sm[ds] : 0;
+    const size_t dyn = PT_DYN_SMEM;
+    if (per_sm == 0) {
+        int coop = 0, dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+        int n = 0;
+        if (coop &&
+            cudaFuncSetAttribute(rq_persist_kernel<FMT, DEQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dyn) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rq_persist_kernel<FMT, DEQ>, PT_THREADS, dyn) ==
+                cudaSuccess &&
+            n > 0)
+            per_sm = n;
+        else
+            per_sm = -1;
+        cudaGetLastError();                          // a refused attribute is not this call's error
+        if (ds >= 0) ctas_per_sm[ds] = per_sm;
+    }
+    if (per_sm <= 0) return cudaSuccess;
+    const int64_t grid = std::min<int64_t>((int64_t)per_sm * sm_count_cached(), 1184);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(PT_THREADS);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, rq_persist_kernel<FMT, DEQ>, pt);
+    launched = e == cudaSuccess;
+    if (!launched) cudaGetLastError();               // e.g. the device is shared: the two passes run instead
+    return cudaSuccess;
+}
+
 template <int FMT, bool DEQ>
 static cudaError_t rq_tensor_t(const QuantArgs& a, cudaStream_t st) {
     RQParams p{};
@@ -846,6 +1113,23 @@ static cudaError_t rq_tensor_t(const QuantArgs& a, cudaStream_t st) {
     if (nvec <= (int64_t)SMALL_THREADS * SMALL_VPT) {
         rq_small_tensor_kernel<FMT, DEQ><<<1, SMALL_THREADS, 0, st>>>(p);
         return cudaGetLastError();
+    }
+    if (p.n >= PT_MIN_ELEMS && (reinterpret_cast<uintptr_t>(a.partials) & 7u) == 0) {
+        PTParams pt{};
+        pt.x = a.x;
+        pt.nvec = nvec;
+        pt.q = a.q;
+        pt.scale = static_cast<float*>(a.scale);
+        pt.deq = a.deq;
+        pt.status = a.status;
+        pt.epoch = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.partials) + kEpochOffset);
+        pt.slots = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(a.partials) + kSlotsOffset);
+        pt.ring = a.hist_ring;
+        pt.slot = p.slot;
+        pt.wait_ns = wait_limit_ns();
+        bool launched = false;
+        launch_persist<FMT, DEQ>(pt, st, launched);
+        if (launched) return cudaSuccess;
     }
     rq_amax_kernel<8><<<(unsigned)grid, QT, 0, st>>>(p);
     p.npartials = (int32_t)grid;

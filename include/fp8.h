@@ -123,8 +123,13 @@ FP8_API int32_t fp8_device_check(void);
 /*
  * Workspace bytes an entry point needs.  which: 0 = fp8_quantize,
  * 1 = fp8_scaled_gemm, 2 = fp8_linear_forward.  For 0, (M, K) is the input
- * shape [rows, cols] and N is ignored.  The workspace needs no initialisation
- * and holds nothing between calls.
+ * shape [rows, cols] and N is ignored.  The workspace needs no initialisation.
+ * For per-tensor current scaling of a large dense tensor (>= 16 Mi elements) the
+ * quantize runs as one cooperative launch whose CTAs exchange their amax through
+ * the workspace; the workspace then keeps a call counter from one call to the next
+ * (nothing else), so calls that share one workspace must not overlap on the GPU,
+ * and after a call that reported FP8_ERR_TIMEOUT its contents are undefined until
+ * the caller zeroes it.
  */
 FP8_API size_t fp8_workspace_size(int32_t which, int64_t M, int64_t N, int64_t K, int32_t mode);
 
@@ -142,9 +147,11 @@ FP8_API size_t fp8_workspace_size(int32_t which, int64_t M, int64_t N, int64_t K
  *   scale_dev    scale buffer in the layout listed with fp8_scaling_t.
  *   hist         host struct, DELAYED only (else NULL); its step is advanced.
  *   dequant_dev  nullable; bf16 [rows, cols] dense, bf16_RNE(fp32(decode(q) * s)).
- *   dev_status   nullable device int32 (FP8_ERR_NONFINITE).
+ *   dev_status   nullable device int32 (FP8_ERR_NONFINITE; FP8_ERR_TIMEOUT if the
+ *                grid-wide amax exchange of the single-launch per-tensor kernel gave up).
  *   workspace_dev, ws_bytes  at least fp8_workspace_size(0, rows, 0, cols, mode) bytes
- *                (0 for modes other than TENSOR/DELAYED).
+ *                (0 for modes other than TENSOR/DELAYED); 8-byte aligned for the
+ *                single-launch per-tensor kernel (otherwise two passes run instead).
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, WORKSPACE, CUDA.
  */
 FP8_API int32_t fp8_quantize(const void* x_dev, int64_t rows, int64_t cols, int64_t ld,

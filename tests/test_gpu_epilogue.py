@@ -241,7 +241,7 @@ def test_rowscale_epilogue(M, N, K, am, bm, yq_fmt):
     check_epilogue(x, w, am, bm, yq_fmt=yq_fmt, seed=M, what=f"rowscale {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (130, 264, 1024)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (130, 264, 1024), (300, 264, 512), (512, 384, 256)])
 def test_block_epilogue(M, N, K):
     x = rand_bf16((M, K), seed=M * 3 + K, spread=1.0)
     w = rand_bf16((N, K), seed=N * 3 + K, std=0.02)
@@ -262,7 +262,7 @@ def test_epilogue_ragged_fp8_stride_and_offset():
     check_epilogue(x, w, R, R, ldq=203, yq_offset=5, what="ragged ldq")
 
 
-@pytest.mark.parametrize("am,bm,M", [(T, T, 64), (T, T, 300), (B1, B128, 128), (MX, MX, 128)])
+@pytest.mark.parametrize("am,bm,M", [(T, T, 64), (T, T, 300), (B1, B128, 128), (B1, B128, 384), (MX, MX, 128)])
 def test_epilogue_exact_integer(am, bm, M):
     """Small-integer codes, unit scales and an integer bias: y, amax and the FP8 output
     codes are exact, so they must equal the oracle bit for bit."""

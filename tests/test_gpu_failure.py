@@ -60,7 +60,8 @@ def test_bounded_wait_runs_out_then_device_recovers(kind, M, N):
     finally:
         fp8.fp8_testing_set_wait_limit_ns(0)
     assert int(status.item()) == fp8.FP8_ERR_TIMEOUT, f"{kind}: status {int(status.item())}"
-    # the context is intact: the same call at the default limit is correct
+    # the context is intact: the same kernel at the default limit is correct
+    qa, sa, qb, sb = _operands(M, N, 1024, seed=M + N + 1)
     status.zero_()
     y = _run(kind, qa, sa, qb, sb, M, N, status)
     assert int(status.item()) == 0

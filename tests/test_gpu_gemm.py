@@ -94,7 +94,8 @@ def test_rowscale_e5m2_operands(fa, fb):
     check_full(x, w, R, R, fa=fa, fb=fb, what=f"formats {fa}/{fb}")
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (130, 260, 1040), (257, 520, 2048), (64, 128, 128)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (130, 260, 1040), (257, 520, 2048), (64, 128, 128),
+                                   (256, 128, 128), (300, 384, 640), (513, 200, 1024), (1024, 1152, 512)])
 def test_block_scaled_shapes(M, N, K):
     g = np.random.default_rng(M + K)
     x = g.standard_normal((M, K)).astype(np.float32)

@@ -436,3 +436,83 @@ def test_cast_exhaustive_every_finite_bf16_pattern(mode):
     x = _exhaustive_rows(amax) if mode == fp8.FP8_SCALE_ROW else _exhaustive_blocks(amax)
     for fmt in FMTS:
         check_parity(x, fmt, mode, dequant=True, what=f"exhaustive mode {mode} fmt {fmt}")
+
+
+# ---------------------------------------------------------------- per-tensor in one launch
+def _per_tensor_run(x_dev, fmt, ws, dequant=True):
+    rows, cols = x_dev.shape
+    q, s, d = fp8.empty_quant_outputs(rows, cols, fp8.FP8_SCALE_TENSOR, dequant=dequant)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8.fp8_quantize(x_dev, fmt, fp8.FP8_SCALE_TENSOR, q, s, dequant=d, dev_status=st, workspace=ws)
+    torch.cuda.synchronize()
+    return q, s, d, int(st.item())
+
+
+def _check_against_oracle(x, q, s, d, fmt, what):
+    rq, rs, rd = oracle.quantize(x, fmt, oracle.TENSOR, dequant=d is not None)
+    assert s.cpu().numpy().view(np.uint32)[0] == rs.view(np.uint32)[0], f"{what}: scale"
+    assert first_mismatch(q.cpu().numpy(), rq) is None, f"{what}: codes"
+    if d is not None:
+        assert first_mismatch(to_host_u16(d), rd) is None, f"{what}: dequant"
+
+
+@pytest.mark.parametrize("shape", [(2048, 8192),      # 16 Mi elements: every CTA region fits on chip
+                                   (2049, 8208),      # just above, ragged CTA regions
+                                   (6000, 4096)])     # a spill part in every region
+def test_per_tensor_single_launch_sizes(shape):
+    """Dense per-tensor tensors from 16 Mi elements take the single-launch kernel (shared
+    memory + registers + re-read spill, one grid-wide amax exchange); bit-exact with the
+    oracle in both formats, codes + scale + dequant."""
+    x = mixed_input(*shape, seed=shape[0])
+    xd = to_dev_bf16(x)
+    ws = fp8.workspace_for(0, shape[0], 0, shape[1], fp8.FP8_SCALE_TENSOR)
+    for fmt in FMTS:
+        q, s, d, st = _per_tensor_run(xd, fmt, ws)
+        assert st == 0
+        _check_against_oracle(x, q, s, d, fmt, f"single launch {shape} fmt {fmt}")
+
+
+def test_per_tensor_single_launch_garbage_workspace_and_repeats():
+    """The workspace needs no initialisation: filled with random bytes first, then reused
+    by calls on changing inputs, the results stay bit-exact (each call's exchange only
+    accepts slots tagged with its own call number)."""
+    rows, cols = 4096, 4096
+    n = fp8.fp8_workspace_size(0, rows, 0, cols, fp8.FP8_SCALE_TENSOR)
+    ws = torch.randint(0, 256, (n,), dtype=torch.uint8, device="cuda")
+    for i in range(4):
+        x = mixed_input(rows, cols, seed=500 + i)
+        if i == 2:
+            x[17, 33] = 0x4F00            # a much larger amax than the calls before
+        q, s, d, st = _per_tensor_run(to_dev_bf16(x), fp8.FP8_E4M3, ws)
+        assert st == 0
+        _check_against_oracle(x, q, s, d, fp8.FP8_E4M3, f"call {i}")
+
+
+def test_per_tensor_single_launch_exchange_timeout_then_recovers():
+    """A 1 ns limit makes the grid-wide exchange run out (every CTA but the last to arrive
+    waits): FP8_ERR_TIMEOUT, no fault; after zeroing the workspace the same call at the
+    default limit is bit-exact."""
+    x = mixed_input(8192, 8192, seed=77)
+    xd = to_dev_bf16(x)
+    ws = fp8.workspace_for(0, 8192, 0, 8192, fp8.FP8_SCALE_TENSOR)
+    seen = []
+    fp8.fp8_testing_set_wait_limit_ns(1)
+    try:
+        for _ in range(3):
+            seen.append(_per_tensor_run(xd, fp8.FP8_E4M3, ws)[3])
+            if seen[-1] == fp8.FP8_ERR_TIMEOUT:
+                break
+    finally:
+        fp8.fp8_testing_set_wait_limit_ns(0)
+    assert fp8.FP8_ERR_TIMEOUT in seen, seen
+    assert set(seen) <= {0, fp8.FP8_ERR_TIMEOUT}
+    ws.zero_()
+    q, s, d, st = _per_tensor_run(xd, fp8.FP8_E4M3, ws)
+    assert st == 0
+    _check_against_oracle(x, q, s, d, fp8.FP8_E4M3, "after the timeout")
+
+
+def test_delayed_step0_single_launch_records_amax():
+    """Step 0 of a large delayed history runs the single-launch kernel and records amax_0."""
+    xs = [inputs.delayed_step_input(t, M=4096, K=8192) for t in range(3)]
+    run_delayed_sequence(xs, fp8.FP8_E4M3, hist_len=4)
