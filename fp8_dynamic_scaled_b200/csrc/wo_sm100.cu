@@ -12,11 +12,14 @@
 //     stages of 3 K blocks loaded as 64-/16-row boxes issued row group by row group;
 //     every FP8 code is read from HBM once;
 //   - eight converter warps turn each 128-row x 64-element half of a K block into
-//     BF16 (exact: every E4M3 and E5M2 value is a BF16 value) and write it in the
-//     K-major 128-byte-swizzled layout the tensor core reads, into a two-slot ring;
-//   - the MMA warp issues tcgen05.mma kind::f16 with the weight as A (M = 128 rows)
-//     and the tokens as B (N = M rounded up to 16, X tiles loaded by TMA as BF16),
-//     FP32 accumulators double-buffered in TMEM across chunks;
+//     BF16 (exact: every E4M3 and E5M2 value is a BF16 value) and store it straight into
+//     tensor memory (tcgen05.st: TMEM lane = weight row, two BF16 per 32-bit column),
+//     into a ring of WO_SLOTS 32-column slots, so the BF16 weight never goes through
+//     shared memory;
+//   - the MMA warp issues tcgen05.mma kind::f16 with the weight as A read from TMEM
+//     (M = 128 rows) and the tokens as B (N = M rounded up to 16, X tiles loaded by TMA
+//     as BF16 into shared memory), FP32 accumulators double-buffered in TMEM across
+//     chunks;
 //   - the epilogue warp of a TMEM lane quarter owns 32 weight rows and writes
 //     bf16(acc * s_w[n]) for every token.
 // Every wait is bounded as in the other kernels.
@@ -34,12 +37,13 @@ constexpr int WO_UNIT = 16;                          // rows of W per work unit
 constexpr int WO_TILE = 128;                         // rows of W per MMA
 constexpr int WO_KBS = 3;                            // K blocks (128 codes) per stage
 constexpr int WO_MAX_STAGES = 4;
-constexpr int WO_SLOTS = 2;                          // BF16 weight ring
+constexpr int WO_SLOTS = 8;                          // BF16 weight ring in TMEM (32 columns a slot)
+constexpr uint32_t WO_ACC_COLS = 128;                // TMEM columns 0-127: two accumulators of <= 64
+constexpr uint32_t WO_TMEM_COLS = 512;
 constexpr int WO_CONV_WARPS = 8, WO_EPI_WARPS = 4;
 constexpr int WO_FIRST_CONV = 2, WO_FIRST_EPI = WO_FIRST_CONV + WO_CONV_WARPS;
 constexpr int WO_THREADS = 32 * (WO_FIRST_EPI + WO_EPI_WARPS);     // 448
 constexpr uint32_t WO_W8_BYTES = WO_TILE * BK;       // 16 KB: FP8 codes of one K block
-constexpr uint32_t WO_HALF_BYTES = WO_TILE * 128;    // 16 KB: 64 BF16 values of 128 rows
 constexpr uint32_t WO_BAR_BYTES = 1024;
 constexpr uint32_t WO_SMEM = 227 * 1024;
 
@@ -48,7 +52,6 @@ struct WoParams {
     int32_t nt;             // tokens per MMA: M rounded up to 16
     int32_t stages;
     uint32_t stage_bytes;   // WO_KBS * (WO_W8_BYTES + 2 * nt * 128)
-    uint32_t ring_off;      // the BF16 weight ring, from the start of the stages
 };
 
 struct WoRange {
@@ -71,11 +74,11 @@ __device__ __forceinline__ void wo_chunk(const WoRange& r, int32_t j, int32_t& n
     w = (ub - ua) * WO_UNIT;
 }
 
-// 16 FP8 codes (one 16-byte chunk) -> 16 BF16 values (two 16-byte chunks), exact.
+// 16 FP8 codes (one 16-byte chunk) -> 16 BF16 values packed two per word (element 2i
+// in the low half of word i), exact.
 template <int WFMT>
-__device__ __forceinline__ void codes16_to_bf16(const uint4& c, uint4& lo, uint4& hi) {
+__device__ __forceinline__ void codes16_to_bf16(const uint4& c, uint32_t* o) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float2 a = decode_pair<WFMT>(w[i] & 0xFFFFu);
@@ -83,8 +86,6 @@ __device__ __forceinline__ void codes16_to_bf16(const uint4& c, uint4& lo, uint4
         o[2 * i] = pack_bf16x2(a.x, a.y);
         o[2 * i + 1] = pack_bf16x2(b.x, b.y);
     }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 template <int WFMT>
@@ -95,16 +96,15 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + WO_MAX_STAGES;
-    uint64_t* bfull = empty + WO_MAX_STAGES;
-    uint64_t* bempty = bfull + WO_SLOTS;
-    uint64_t* tfull = bempty + WO_SLOTS;
+    uint64_t* afull = empty + WO_MAX_STAGES;           // a BF16 slot is written (converters)
+    uint64_t* aempty = afull + WO_SLOTS;               // its MMAs are done (commit)
+    uint64_t* tfull = aempty + WO_SLOTS;
     uint64_t* tempty = tfull + 2;
     uint64_t* teardown = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
     // stage s: FP8 W of WO_KBS K blocks (16 KB each), then X as 2 * WO_KBS BF16 halves
     uint8_t* stages = smem + WO_BAR_BYTES;
-    uint8_t* ring = stages + d.ring_off;                 // WO_SLOTS x 16 KB of BF16 weight
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -117,11 +117,13 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], 1);
+            // the stage is free once the converters have read its W codes and the MMAs
+            // its X tiles
+            ptx::mbar_init(&empty[s], WO_CONV_WARPS + 1);
         }
         for (int t = 0; t < WO_SLOTS; ++t) {
-            ptx::mbar_init(&bfull[t], WO_CONV_WARPS);
-            ptx::mbar_init(&bempty[t], 1);
+            ptx::mbar_init(&afull[t], WO_CONV_WARPS);
+            ptx::mbar_init(&aempty[t], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&tfull[b], 1);
@@ -135,7 +137,7 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         ptx::prefetch_tmap(&tmW16);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_alloc(tmem_slot, WO_TMEM_COLS);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -179,7 +181,7 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         // ------------------------------------------------ MMA issuer: D[n, m] += W_bf16 X^T
         uint32_t stage = 0, phase = 0, acc_it = 0, conv_it = 0;
         bool ok = true;
-        const uint32_t s0 = ptx::smem_u32(stages), r0 = ptx::smem_u32(ring);
+        const uint32_t s0 = ptx::smem_u32(stages);
         for (int32_t j = 0; j < range.nch && ok; ++j) {
             const uint32_t buf = acc_it & 1u, use = acc_it >> 1;
             if (!wait_bounded(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
@@ -190,22 +192,22 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 const uint32_t sx = s0 + stage * d.stage_bytes + x_off;
                 for (int32_t hb = 0; hb < 2 * kbs; ++hb) {
                     const uint32_t t = conv_it % WO_SLOTS, tu = conv_it / WO_SLOTS;
-                    if (!wait_bounded(&bfull[t], tu & 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+                    if (!wait_bounded(&afull[t], tu & 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
                     ptx::tc_fence_after();
                     if (lane == 0) {
+                        const uint32_t a0 = tmem_base + WO_ACC_COLS + t * 32;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {                       // K = 16 BF16 per instruction
-                            const uint64_t ad = ptx::sdesc_kmajor_sw128(r0 + t * WO_HALF_BYTES + k * 32);
                             const uint64_t bd = ptx::sdesc_kmajor_sw128(sx + hb * x_half + k * 32);
-                            ptx::mma_f16(tmem_base + buf * 64, ad, bd, p.idesc, (kc | hb | k) != 0);
+                            ptx::mma_f16_ts(tmem_base + buf * 64, a0 + k * 8, bd, p.idesc, (kc | hb | k) != 0);
                         }
-                        ptx::mma_commit(&bempty[t]);
+                        ptx::mma_commit(&aempty[t]);
                     }
                     __syncwarp();
                     ++conv_it;
                 }
                 if (!ok) break;
-                if (lane == 0) ptx::mma_commit(&empty[stage]);
+                if (lane == 0) ptx::mma_commit(&empty[stage]);      // its X tiles are read
                 __syncwarp();
                 if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
             }
@@ -220,11 +222,15 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
         __syncwarp();
     } else if (warp < WO_FIRST_EPI) {
-        // ------------------------------------------------ converters: FP8 -> BF16 tiles
-        // thread ct owns row (ct % 128) and one half (ct / 128) of that row's 64 values
-        const int ct = threadIdx.x - 32 * WO_FIRST_CONV;
-        const int row = ct & 127, part = ct >> 7;
+        // ------------------------------------------------ converters: FP8 -> BF16 in TMEM
+        // warp cw owns the 32 weight rows of its TMEM lane quarter and one 32-value part of
+        // each 64-value half K block: 32 codes a thread -> 16 words -> one 16-column store
+        const int cw = warp - WO_FIRST_CONV;                 // 0 .. 7
+        const int quarter = warp & 3;                        // TMEM lane quarter of this warp
+        const int part = cw >> 2;                            // 32-value part of a half K block
+        const int row = quarter * 32 + lane;
         const int sw = row & 7;                              // the row's 128-byte swizzle phase
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         uint32_t stage = 0, phase = 0, conv_it = 0;
         bool ok = true;
         for (int32_t j = 0; j < range.nch && ok; ++j) {
@@ -234,24 +240,26 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 const uint8_t* w8 = stages + stage * d.stage_bytes;
                 for (int32_t hb = 0; hb < 2 * kbs; ++hb) {
                     const uint32_t t = conv_it % WO_SLOTS, tu = conv_it / WO_SLOTS;
-                    if (!wait_bounded(&bempty[t], (tu & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+                    if (!wait_bounded(&aempty[t], (tu & 1u) ^ 1u, abort_flag, p.status, p.wait_ns)) { ok = false; break; }
+                    ptx::tc_fence_after();
                     const int b = hb >> 1, h = hb & 1;
                     const uint8_t* src = w8 + b * WO_W8_BYTES + row * 128;
-                    uint8_t* dst = ring + t * WO_HALF_BYTES + row * 128;
+                    uint32_t o[16];
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
-                        const int jj = 2 * part + q;                 // 16-code chunk within this half
-                        const uint4 c = *reinterpret_cast<const uint4*>(src + (((4 * h + jj) ^ sw) * 16));
-                        uint4 lo, hi;
-                        codes16_to_bf16<WFMT>(c, lo, hi);
-                        *reinterpret_cast<uint4*>(dst + (((2 * jj) ^ sw) * 16)) = lo;
-                        *reinterpret_cast<uint4*>(dst + (((2 * jj + 1) ^ sw) * 16)) = hi;
+                        const int jj = 4 * h + 2 * part + q;          // 16-code chunk of the 128-byte row
+                        codes16_to_bf16<WFMT>(*reinterpret_cast<const uint4*>(src + ((jj ^ sw) * 16)), o + 8 * q);
                     }
-                    ptx::fence_proxy_async_smem();               // generic writes -> tensor-core reads
+                    ptx::tmem_st_32x32b_x16(tmem_base + lane_base + WO_ACC_COLS + t * 32 + part * 16, o);
+                    ptx::tmem_st_wait();
+                    ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&bfull[t]);
+                    if (lane == 0) ptx::mbar_arrive(&afull[t]);
                     ++conv_it;
                 }
+                if (!ok) break;
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&empty[stage]);     // its W codes are read
                 if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
             }
         }
@@ -294,7 +302,7 @@ fp8_wo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 1) ptx::tmem_dealloc(tmem_base, 128);
+    if (warp == 1) ptx::tmem_dealloc(tmem_base, WO_TMEM_COLS);
 }
 
 template <int WFMT>
@@ -314,9 +322,7 @@ static cudaError_t launch_wo_t(const WoArgs& g, cudaStream_t st) {
     d.nt = (int32_t)((g.M + 15) / 16 * 16);
     d.units = (int32_t)((g.N + WO_UNIT - 1) / WO_UNIT);
     d.stage_bytes = WO_KBS * (WO_W8_BYTES + 2u * (uint32_t)d.nt * 128);
-    d.stages = (int32_t)std::min<uint32_t>(
-        WO_MAX_STAGES, (WO_SMEM - 1024 - WO_BAR_BYTES - WO_SLOTS * WO_HALF_BYTES) / d.stage_bytes);
-    d.ring_off = (uint32_t)d.stages * d.stage_bytes;
+    d.stages = (int32_t)std::min<uint32_t>(WO_MAX_STAGES, (WO_SMEM - 1024 - WO_BAR_BYTES) / d.stage_bytes);
     // BF16 x BF16 (kind::f16: formats 1 = BF16 in bits 7-9 and 10-12), FP32 D, M = 128, N = nt
     p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(d.nt >> 3) << 17) | ((uint32_t)(WO_TILE >> 4) << 24);
     CUtensorMap tx, t64, t16;
@@ -335,7 +341,7 @@ static cudaError_t launch_wo_t(const WoArgs& g, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         if (ds >= 0) attr_done[ds] = true;
     }
-    const uint32_t smem = 1024 + WO_BAR_BYTES + d.ring_off + WO_SLOTS * WO_HALF_BYTES;
+    const uint32_t smem = 1024 + WO_BAR_BYTES + (uint32_t)d.stages * d.stage_bytes;
     const int grid = std::max(1, std::min(d.units, num_sms()));
     fp8_wo_kernel<WFMT><<<grid, WO_THREADS, smem, st>>>(tx, t64, t16, p, d);
     return cudaGetLastError();
