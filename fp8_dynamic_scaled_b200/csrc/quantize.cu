@@ -805,7 +805,7 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const
 // before (a stale or uninitialised slot would also have to match a 16-bit check of its
 // tag and CTA).  CUDA-graph replays advance E the same way.
 constexpr int PT_THREADS = 512;
-constexpr int PT_REG_VEC = 16;                      // 16-byte vectors per thread kept in registers
+constexpr int PT_REG_VEC = 20;                      // 16-byte vectors per thread kept in registers
 constexpr uint32_t PT_HELD_BYTES = 96 * 1024;       // bytes per CTA kept in shared memory
 constexpr int PT_HELD_CHUNKS = 6;                   // its bulk copies (one mbarrier each)
 constexpr int PT_RING = 4;                          // spill ring slots

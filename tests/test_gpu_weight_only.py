@@ -134,3 +134,33 @@ def test_weight_only_llama70b_layer_full_size(M):
     cols = np.sort(np.random.default_rng(5).choice(qw.shape[0], 2048, replace=False))
     y_ref, bound = oracle.weight_only_ref(x, qw[cols], sw[cols], R, E4M3)
     assert_gemm_close(y[:, cols], y_ref, bound, f"weight-only llama70b M={M}")
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 16, 64])
+def test_weight_only_every_code_decodes_exactly(M, fmt):
+    """Every one of the 256 codes through the weight decode of both kernels.  X is one-hot
+    (token m picks column m), so y[m, n] is the decoded code w[n, m] itself, exact in
+    bf16 (every FP8 value is a bf16 value): the finite codes fill rows M codes a row,
+    subnormals and both zeros included, and are compared bit for bit with the oracle's
+    decode table.  A NaN or Inf code (E5M2 also has Inf) gets a row of its own at column
+    0: token 0 reads the code times 1, every other token 0 times the code (NaN)."""
+    table = oracle.decode_table(fmt)
+    codes = np.arange(256)
+    finite = codes[np.isfinite(table)]
+    special = codes[~np.isfinite(table)]
+    K = max(64, -(-M // 16) * 16)
+    nf = -(-len(finite) // M)
+    w = np.zeros((nf + len(special), K), np.uint8)
+    flat = np.zeros(nf * M, np.int64)
+    flat[:len(finite)] = finite
+    w[:nf, :M] = flat.reshape(nf, M)
+    w[nf:, 0] = special
+    x = np.zeros((M, K), np.float32)
+    x[np.arange(M), np.arange(M)] = 1.0
+    y = bf16_bits_to_f64(run_wo(inputs.bf16_bits(x), w, np.ones(1, np.float32), T, fmt))
+    want = table[w[:nf, :M]].T                       # [M, nf]
+    assert np.array_equal(y[:, :nf], want), f"finite codes, fmt {fmt}, M {M}"
+    got_s = y[:, nf:]
+    assert np.array_equal(got_s[0], table[special], equal_nan=True), f"special codes, token 0, fmt {fmt}"
+    assert np.all(np.isnan(got_s[1:])), f"special codes times 0, fmt {fmt}"
