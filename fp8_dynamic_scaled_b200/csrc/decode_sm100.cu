@@ -23,8 +23,9 @@
 //   - X comes as one box per K block of the rounded-up token count (rows past M are
 //     zero-filled by TMA); FP32 accumulators are double-buffered in TMEM across
 //     chunks;
-//   - the epilogue warp of each TMEM lane quarter holds 32 weight rows: for every
-//     token it writes 32 consecutive outputs of Y's row (a 64-byte store per warp).
+//   - the two epilogue warps of each TMEM lane quarter hold its 32 weight rows and
+//     split the tokens in groups of 16: for each of its tokens a warp writes 32
+//     consecutive outputs of Y's row (a 64-byte store per warp).
 // Hopper-era decode kernels split K across CTAs (and reduce the partial sums) to
 // occupy the machine; with per-SM ranges of whole rows W is read exactly once.
 // Every wait is bounded as in the tiled kernels.
@@ -70,11 +71,14 @@ __device__ __forceinline__ void decode_chunk(const DecodeRange& r, int32_t j, in
     w = (ub - ua) * D_UNIT;
 }
 
+constexpr int D_EPI_WARPS = 8;             // two per TMEM lane quarter, each half of the tokens
+constexpr int D_THREADS = 32 * (2 + D_EPI_WARPS);
+
 template <bool EXT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(D_THREADS, 1)
 fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW64,
                   const __grid_constant__ CUtensorMap tmW16, const GemmParams p, const DecodeParams d) {
-    constexpr int EPI_WARPS = 4;
+    constexpr int EPI_WARPS = D_EPI_WARPS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -205,8 +209,10 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue: lane = weight row
+        // two warps per TMEM lane quarter: warp half th takes the 16-token groups th, th + 2, ...
         pdl_wait();                           // X's scales (and epilogue inputs) may be just written
         const int quarter = warp & 3;
+        const int th = (warp - 2) >> 2;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         uint32_t amax_bits = 0;               // |y| as fp32 patterns (order-preserving for y >= 0)
         float ys = 0.0f;
@@ -230,7 +236,7 @@ fp8_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const float sw = valid ? __ldg(p.sb + (int64_t)n * p.sb_stride) : 0.0f;
                 float bias = 0.0f;
                 if (EXT && p.bias && valid) bias = bf16bits_to_float(__ldg(p.bias + n));
-                for (int32_t c0 = 0; c0 < p.M; c0 += 16) {
+                for (int32_t c0 = 16 * th; c0 < p.M; c0 += 32) {
                     uint32_t acc[16];
                     ptx::tmem_ld_32x32b_x16(tmem_base + lane_base + buf * 128 + c0, acc);
                     ptx::tmem_ld_wait();
@@ -309,7 +315,7 @@ static cudaError_t launch_decode_t(const GemmArgs& g, GemmParams p, cudaStream_t
     const int grid = std::max(1, std::min(d.units, num_sms()));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(D_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
