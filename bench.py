@@ -27,6 +27,7 @@ import json
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -108,26 +109,48 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.reader = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.lines.append(line)
+
+    def _wait_lines(self, n: int, limit_s: float):
+        t0 = time.monotonic()
+        while len(self.lines) < n and time.monotonic() - t0 < limit_s and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def __enter__(self):
+        # the sampler is live (its first sample read) before the timed region starts, and
+        # one more sample is read after it ends, so that a region shorter than the 200 ms
+        # period still has samples on both sides
+        self.lines = []
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        self._wait_lines(1, 5.0)
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self.proc is None:
+            return
+        self._wait_lines(len(self.lines) + 1, 1.0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.proc.wait()
+        self.reader.join(timeout=5)
+        self.lines = list(self.lines)
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -460,22 +483,23 @@ def extras(torch, fp8, stream, peaks):
             def run_dec():
                 fp8.fp8_scaled_gemm(xd, xsd, fp8.FP8_SCALE_ROW, fp8.FP8_E4M3, wq, wsc, fp8.FP8_SCALE_ROW,
                                     fp8.FP8_E4M3, yd, stream=stream)
+            # per call: events around each of 50 calls, median; and the 50 calls back to
+            # back between two events (that time also holds any gap between launches)
+            ms, _ = time_kernel(torch, run_dec, 50, stream, warmup=5)
             with torch.cuda.stream(stream):
-                for _ in range(5):
-                    run_dec()
-                torch.cuda.synchronize()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 for _ in range(50):
                     run_dec()
                 b.record(stream)
             torch.cuda.synchronize()
-            ms = a.elapsed_time(b) / 50
+            loop_ms = a.elapsed_time(b) / 50
             nbytes = N * K + Md * K + 4 * (Md + N) + 2 * Md * N
             res[f"M{Md}"] = {"us": ms * 1e3, "GB_per_s": nbytes / (ms * 1e-3) / 1e9,
                              "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
-                             "tflops": 2.0 * Md * N * K / (ms * 1e-3) / 1e12}
-        res["note"] = "N=28672, K=8192 per-row scales; bytes = W codes + X codes + scales + bf16 Y"
+                             "tflops": 2.0 * Md * N * K / (ms * 1e-3) / 1e12, "back_to_back_us": loop_ms * 1e3}
+        res["note"] = ("N=28672, K=8192 per-row scales; bytes = W codes + X codes + scales + bf16 Y; us = median "
+                       "of 50 calls each between two events; back_to_back_us = 50 calls between two events")
         # the whole decode layer: fp8_linear_forward (X quantize, then the GEMM launched as
         # its programmatic dependent, streaming W while X is quantised) against the same
         # two steps as separate calls; interleaved rounds of 50 calls, median round
@@ -763,7 +787,7 @@ def run_quant_sweep(args, torch, fp8, stream, barrier, dist, world, rank, gpu_in
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"],
                          "traffic": profiled_traffic("quant_tensor_quant_sweep"),
-                         "kernel": "rq_amax_kernel + rq_tensor_kernel<CAST> (one fp8_quantize call)",
+                         "kernel": "rq_persist_kernel (one fp8_quantize call: a single cooperative launch)",
                          "peak_source": f"{peak_src} hbm_gbs", "call_us_avg": k_ms * 1e3},
             "clocks": clk.summary(), "gpu_launches": args.steps * 4}
     if rank == 0:
