@@ -313,7 +313,7 @@ def time_kernel(torch, fn, reps, stream, warmup=3):
     return statistics.median(ts), ts[min(len(ts) - 1, int(0.95 * len(ts)))]
 
 
-def extras(torch, fp8, stream, peaks):
+def extras(torch, fp8, stream, peaks, gpu_index=0):
     """Per-config numbers behind the metric (rank 0, one GPU)."""
     from fp8_dynamic_scaled_b200 import inputs
     out = {}
@@ -473,9 +473,15 @@ def extras(torch, fp8, stream, peaks):
     except Exception as ex:
         out["epilogue_options"] = {"error": str(ex)[:200]}
     # decode-shaped calls of the same layer: M tokens against the 235 MB FP8 weight, which
-    # no L2 holds, so every call streams W from HBM; the bound is W's bytes
+    # no L2 holds, so every call streams W from HBM; the bound is W's bytes.  The GEMM loops
+    # just before run the part at its power cap; an idle second lets the clocks come back
+    # before these short calls, and the section records the clocks it saw.
+    clk = ClockSampler(gpu_index)
     try:
         res = {}
+        torch.cuda.synchronize()
+        time.sleep(1.0)
+        clk.__enter__()
         for Md in (1, 8, 16, 32, 64, 128, 256):
             yd = torch.empty((Md, N), dtype=torch.bfloat16, device="cuda")
             xd, xsd = xq[:Md], xs[:Md]
@@ -545,8 +551,11 @@ def extras(torch, fp8, stream, peaks):
             nbytes = N * K + 2 * Md * K + 4 * N + 2 * Md * N
             res[f"weight_only_M{Md}"] = {"us": med * 1e3, "GB_per_s": nbytes / (med * 1e-3) / 1e9,
                                          "frac_of_hbm": nbytes / (med * 1e-3) / 1e9 / hbm}
+        clk.__exit__(None, None, None)
+        res["clocks"] = clk.summary()
         out["decode_shapes"] = res
     except Exception as ex:
+        clk.__exit__(None, None, None)
         out["decode_shapes"] = {"error": str(ex)[:200]}
     xq = wq = y = yq = qy = None      # release the layer's buffers
     torch.cuda.empty_cache()
@@ -936,7 +945,7 @@ def main():
         del wl
         torch.cuda.empty_cache()
         if world == 1 and not args.no_extras:
-            line["configs"] = extras(torch, fp8, stream, peaks)
+            line["configs"] = extras(torch, fp8, stream, peaks, gpu_index)
             line["summary"] = config_summary(line["configs"])
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_line()
