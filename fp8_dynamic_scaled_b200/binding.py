@@ -32,7 +32,7 @@ FP8_ERR_NONFINITE, FP8_ERR_TIMEOUT, FP8_ERR_CUDA, FP8_ERR_WORKSPACE = 4, 5, 6, 7
 EXPORTED = ("fp8_abi_version", "fp8_status_string", "fp8_device_check", "fp8_workspace_size",
             "fp8_quantize", "fp8_scaled_gemm", "fp8_linear_forward", "fp8_linear_forward_noalloc",
             "fp8_amax", "fp8_quantize_with_amax", "fp8_scaled_gemm_ex", "fp8_linear_forward_ex",
-            "fp8_weight_only_linear", "fp8_testing_set_wait_limit_ns")
+            "fp8_weight_only_linear", "fp8_testing_set_wait_limit_ns", "fp8_testing_encode_f32_range")
 FP8_WEIGHT_ONLY_MAX_TOKENS = 64
 FP8_NOALLOC_SCRATCH_BYTES = 4194304
 
@@ -77,6 +77,8 @@ _lib.fp8_weight_only_linear.restype = _I32
 _lib.fp8_weight_only_linear.argtypes = [_P, _I64, _I64, _I64, _P, _P, _I32, _I32, _I64, _P, _I64, _P, _P]
 _lib.fp8_testing_set_wait_limit_ns.restype = None
 _lib.fp8_testing_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.fp8_testing_encode_f32_range.restype = _I32
+_lib.fp8_testing_encode_f32_range.argtypes = [ctypes.c_uint32, _I64, _I32, _P, _P]
 _lib.fp8_linear_forward_noalloc.restype = _I32
 _lib.fp8_linear_forward_noalloc.argtypes = [_P, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(fp8_history_t), _P,
                                             _P, _I32, _I32, _I64, _P, _I64, _P, _P]
@@ -129,6 +131,15 @@ def fp8_device_check() -> int:
 def fp8_testing_set_wait_limit_ns(ns: int) -> None:
     """Testing hook (include/fp8_testing.h): limit of each GEMM pipeline wait; 0 = default."""
     _lib.fp8_testing_set_wait_limit_ns(int(ns))
+
+
+def fp8_testing_encode_f32_range(first_bits: int, q, fmt: int, *, stream=None) -> None:
+    """Testing hook (include/fp8_testing.h): q[i] = encode step of the fp32 value with bit
+    pattern first_bits + i, for every byte of the uint8 device tensor q."""
+    if q.dtype != torch.uint8 or not q.is_contiguous():
+        raise TypeError("q must be a contiguous uint8 tensor")
+    _check(_lib.fp8_testing_encode_f32_range(int(first_bits), q.numel(), fmt, _ptr(q), _stream(stream)),
+           "fp8_testing_encode_f32_range")
 
 
 def fp8_workspace_size(which: int, M: int, N: int, K: int, mode: int) -> int:

@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8.so")
-SOURCES = ["api.cu", "quantize.cu", "gemm_sm100.cu", "decode_sm100.cu", "wo_sm100.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm_sm100.cu", "decode_sm100.cu", "wo_sm100.cu", "noalloc.cu", "testing.cu"]
 HEADERS = ["common.cuh", "gemm_common.cuh", "kernels.h", "ptx.cuh"]
 PUBLIC_HEADERS = [os.path.join(os.path.dirname(HERE), "include", h) for h in ("fp8.h", "fp8_testing.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

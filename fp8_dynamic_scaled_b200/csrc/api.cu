@@ -212,6 +212,16 @@ int32_t fp8_device_check(void) { return device_gate(); }
 
 void fp8_testing_set_wait_limit_ns(uint64_t ns) { set_wait_limit_ns(ns); }
 
+int32_t fp8_testing_encode_f32_range(uint32_t first_bits, int64_t n, int32_t fmt, uint8_t* q, void* stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (n < 0 || (uint64_t)first_bits + (uint64_t)n > ((uint64_t)1 << 32)) return FP8_ERR_INVALID_ARG;
+    if (n == 0) return FP8_OK;
+    if (q == nullptr) return FP8_ERR_INVALID_ARG;
+    const int32_t gate = device_gate();
+    if (gate != FP8_OK) return gate;
+    return cuda_status(launch_encode_f32_range(first_bits, n, fmt, q, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fp8_workspace_size(int32_t which, int64_t M, int64_t N, int64_t K, int32_t mode) {
     (void)N;
     if (which == 0) return (mode == FP8_SCALE_TENSOR || mode == FP8_SCALE_DELAYED) ? partials_bytes() : 0;

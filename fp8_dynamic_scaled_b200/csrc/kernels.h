@@ -74,6 +74,10 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
 void set_wait_limit_ns(uint64_t ns);
 uint64_t wait_limit_ns();
 
+// testing.cu: the n fp32 values with bit patterns first .. first + n - 1 through the
+// encode step of the quantize kernels (n >= 1, first + n <= 2^32, q holds n bytes).
+cudaError_t launch_encode_f32_range(uint32_t first, int64_t n, int32_t fmt, uint8_t* q, cudaStream_t st);
+
 struct WoArgs {              // weight-only FP8 linear (wo_sm100.cu)
     const uint16_t* x;       // bf16 [M, K], row stride ldx
     int64_t ldx;

@@ -722,8 +722,25 @@ void orc_decode_table(int fmt, double* out256) {
 }
 
 /* Vector helpers so the tests can drive large arrays through ctypes. */
+typedef struct {
+    const float* v;
+    float s;
+    int fmt;
+    uint8_t* out;
+} ejob;
+static void encode_range(void* c, int64_t i0, int64_t i1, int part) {
+    const ejob* j = (const ejob*)c;
+    (void)part;
+    for (int64_t i = i0; i < i1; ++i) j->out[i] = orc_encode((double)j->v[i], j->fmt);
+}
+static void quant_scaled_range(void* c, int64_t i0, int64_t i1, int part) {
+    const ejob* j = (const ejob*)c;
+    (void)part;
+    for (int64_t i = i0; i < i1; ++i) j->out[i] = quant_one(j->v[i], j->s, j->fmt, NULL);
+}
 void orc_encode_array(const float* v, int64_t n, int fmt, uint8_t* out) {
-    for (int64_t i = 0; i < n; ++i) out[i] = orc_encode((double)v[i], fmt);
+    ejob j = {v, 1.0f, fmt, out};
+    orc_parallel(n, 4096, &j, encode_range);
 }
 void orc_encode_bruteforce_array(const float* v, int64_t n, int fmt, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = orc_encode_bruteforce((double)v[i], fmt);
@@ -737,5 +754,6 @@ void orc_dequant_scaled_array(const uint8_t* q, int64_t n, float s, int fmt, uin
     for (int64_t i = 0; i < n; ++i) out[i] = dequant_one(q[i], s, fmt);
 }
 void orc_quant_scaled_array(const float* v, int64_t n, float s, int fmt, uint8_t* out) {
-    for (int64_t i = 0; i < n; ++i) out[i] = quant_one(v[i], s, fmt, NULL);
+    ejob j = {v, s, fmt, out};
+    orc_parallel(n, 4096, &j, quant_scaled_range);
 }

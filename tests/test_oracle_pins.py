@@ -512,6 +512,9 @@ def test_results_do_not_depend_on_the_thread_count():
             pm = np.repeat(np.arange(259), 7)
             pn = np.tile(np.arange(0, 140, 20), 259)
             res.append(oracle.gemm_ref_points(qa, sa, oracle.ROW, E4M3, qb, sb, oracle.ROW, E4M3, pm, pn))
+            v = np.arange(0x3B000000, 0x3B000000 + 100003, dtype=np.uint32).view(np.float32)   # ragged ranges
+            res.extend(oracle.encode(v, fmt) for fmt in (E4M3, E5M2))
+            res.extend(oracle.quant_scaled(v, 0.75, fmt) for fmt in (E4M3, E5M2))
             outs[n] = res
         def flat(r):
             out = []
