@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libfp8.so (declared in include/fp8.h): argument checks,
 // device gate, workspace carving and kernel dispatch.  No compute happens here.
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -18,6 +19,20 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// The compute capability major the gate sees instead of the device's own, from the
+// environment variable FP8_B200_FORCE_CC_MAJOR (read once per process), or -1: a test
+// uses it to drive the unsupported-device path on a B200.
+int forced_cc_major() {
+    static const int v = [] {
+        const char* e = std::getenv("FP8_B200_FORCE_CC_MAJOR");
+        if (e == nullptr || *e == '\0') return -1;
+        char* end = nullptr;
+        const long n = std::strtol(e, &end, 10);
+        return (end != e && *end == '\0' && n >= 0 && n < 100) ? (int)n : -1;
+    }();
+    return v;
+}
+
 // FP8_OK when the current device is compute capability 10.x.
 int32_t device_gate() {
     static int cache[kMaxDevices];   // 0 unknown, 1 ok, 2 unsupported
@@ -26,6 +41,7 @@ int32_t device_gate() {
     if (dev >= 0 && dev < kMaxDevices && cache[dev] != 0) return cache[dev] == 1 ? FP8_OK : FP8_ERR_UNSUPPORTED_DEVICE;
     int major = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FP8_ERR_CUDA;
+    if (forced_cc_major() >= 0) major = forced_cc_major();
     const int ok = major == 10 ? 1 : 2;
     if (dev >= 0 && dev < kMaxDevices) cache[dev] = ok;
     return ok == 1 ? FP8_OK : FP8_ERR_UNSUPPORTED_DEVICE;

@@ -117,7 +117,10 @@ FP8_API const char* fp8_status_string(int32_t status);
 
 /* FP8_OK when the current CUDA device is compute capability 10.x (sm_100a),
  * FP8_ERR_UNSUPPORTED_DEVICE otherwise, FP8_ERR_CUDA when CUDA is unusable.
- * (The device gate of [FRLP] section "5.2" preflight, moved to the library.) */
+ * (The device gate of [FRLP] section "5.2" preflight, moved to the library.)  Every
+ * entry point that launches work applies the same gate first.  For tests, the
+ * environment variable FP8_B200_FORCE_CC_MAJOR (a decimal number, read once per
+ * process) replaces the device's compute capability major in the gate. */
 FP8_API int32_t fp8_device_check(void);
 
 /*
