@@ -580,6 +580,18 @@ def extras(torch, fp8, stream, peaks, gpu_index=0):
     host_us = (time.perf_counter() - t0) / 200 * 1e6
     torch.cuda.synchronize()
     out["linear_small"] = {"us_median": med * 1e3, "us_p95": p95 * 1e3, "host_us_per_call": host_us}
+    # the same call captured once in a CUDA graph (the calls allocate nothing and run on
+    # the given stream) and replayed: the launch path without the per-call host work
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            fp8.fp8_linear_forward(x, fp8.FP8_E4M3, fp8.FP8_SCALE_TENSOR, wq, wsc, fp8.FP8_SCALE_TENSOR,
+                                   fp8.FP8_E4M3, y, lws, stream=stream)
+        gmed, gp95 = time_kernel(torch, g.replay, 100, stream)
+        out["linear_small"].update({"graph_replay_us_median": gmed * 1e3, "graph_replay_us_p95": gp95 * 1e3})
+        del g
+    except Exception as ex:
+        out["linear_small"]["graph_replay_error"] = str(ex)[:200]
     return out
 
 
@@ -609,6 +621,7 @@ def config_summary(cfg):
     pick("decode_M64_frac_hbm", "decode_shapes", "M64", "frac_of_hbm")
     pick("weight_only_M16_us", "decode_shapes", "weight_only_M16", "us")
     pick("linear_small_us", "linear_small", "us_median")
+    pick("linear_small_graph_us", "linear_small", "graph_replay_us_median")
     return out
 
 
