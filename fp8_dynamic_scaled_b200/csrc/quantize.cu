@@ -785,9 +785,11 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) rq_small_tensor_kernel(const
 // kernels above read X twice.  This kernel runs one CTA per SM, all resident at once (a
 // cooperative launch), in two phases around one grid-wide exchange of the amax:
 //   own   each CTA owns one contiguous piece of X at the front of the tensor: the first
-//         PT_HELD_BYTES of it are bulk-copied into shared memory, the rest (up to
-//         PT_THREADS * PT_REG_VEC vectors) loaded into registers; both stay on chip
-//         across the exchange;
+//         PT_HELD_BYTES of it are bulk-copied into shared memory, the next (up to
+//         PT_THREADS * PT_REG_VEC vectors) loaded into registers, the rest (up to
+//         PT_THREADS * PT_TMEM_VEC vectors) loaded and stored into tensor memory (all
+//         512 columns; warp w owns a 128-column group of its lane quarter w % 4); all
+//         three stay on chip across the exchange;
 //   spill the rest of X, in chunks of PT_SLOT_BYTES dealt round-robin to the CTAs
 //         (chunk c to CTA c mod G, so every CTA's share is spread over the whole tensor),
 //         streamed through a ring of shared-memory slots filled by bulk copies (many
@@ -811,7 +813,10 @@ constexpr int PT_HELD_CHUNKS = 6;                   // its bulk copies (one mbar
 constexpr int PT_RING = 4;                          // spill ring slots
 constexpr uint32_t PT_SLOT_BYTES = 24 * 1024;       // bytes per slot: 3 vectors per thread
 constexpr int64_t PT_SLOT_VEC = PT_SLOT_BYTES / 16;
-constexpr int64_t PT_OWN_VEC = PT_HELD_BYTES / 16 + (int64_t)PT_THREADS * PT_REG_VEC;
+constexpr int PT_TMEM_VEC = 32;                      // 16-byte vectors per thread kept in tensor memory
+constexpr int PT_TMEM_BATCH = 4;                     // vectors a thread moves per tcgen05.st / ld
+constexpr uint32_t PT_TMEM_COLS = 512;               // all of TMEM: 128 lanes x 512 columns = 256 KB
+constexpr int64_t PT_OWN_VEC = PT_HELD_BYTES / 16 + (int64_t)PT_THREADS * (PT_REG_VEC + PT_TMEM_VEC);
 constexpr uint32_t PT_DYN_SMEM = PT_HELD_BYTES + PT_RING * PT_SLOT_BYTES + 8 * (PT_HELD_CHUNKS + PT_RING);
 constexpr int64_t PT_MIN_ELEMS = (int64_t)16 << 20; // smaller tensors: the two-pass kernels (L2 holds X)
 
@@ -855,12 +860,18 @@ __global__ void __launch_bounds__(PT_THREADS, 1) rq_persist_kernel(const PTParam
     uint64_t* rbar = hbar + PT_HELD_CHUNKS;
     __shared__ uint32_t red[32];
     __shared__ uint32_t s_epoch;
+    __shared__ uint32_t s_tmem;
     const int t = threadIdx.x;
     const int64_t G = gridDim.x, b = blockIdx.x;
-    // this CTA's own piece [v0, v1): held part [v0, r0), registers [r0, v1)
+    // this CTA's own piece [v0, v1): held part [v0, r0), registers [r0, r1), tensor memory
+    // [r1, v1); thread t's j-th vector of the last two is r0 + t + PT_THREADS j (r1 + ...)
     const int64_t v0 = min(p.nvec, b * PT_OWN_VEC), v1 = min(p.nvec, v0 + PT_OWN_VEC);
     const int64_t n_held = min(v1 - v0, (int64_t)(PT_HELD_BYTES / 16));
     const int64_t r0 = v0 + n_held;
+    const int64_t r1 = min(v1, r0 + (int64_t)PT_THREADS * PT_REG_VEC);
+    const int warp = t >> 5;
+    // this thread's TMEM words: lane (warp % 4) * 32 + lane, columns from (warp / 4) * 128
+    const uint32_t tm_off = ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * 128u;
     // the spill: everything past the own pieces, in chunks of PT_SLOT_VEC vectors
     const int64_t sp0 = min(p.nvec, G * PT_OWN_VEC);
     const int64_t nsc = (p.nvec - sp0 + PT_SLOT_VEC - 1) / PT_SLOT_VEC;
@@ -878,7 +889,14 @@ __global__ void __launch_bounds__(PT_THREADS, 1) rq_persist_kernel(const PTParam
         for (int c = 0; c < PT_HELD_CHUNKS + PT_RING; ++c) ptx::mbar_init(&hbar[c], 1);
         ptx::fence_mbar_init();
     }
-    __syncthreads();                                   // the barriers and s_epoch are set
+    if (warp == 0) {                                   // one CTA per SM: all of TMEM is free
+        ptx::tmem_alloc(&s_tmem, PT_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();                                   // the barriers, s_epoch and s_tmem are set
+    ptx::tc_fence_after();
+    const uint32_t tmem = s_tmem + tm_off;
     const uint32_t tag = s_epoch + 1u;
     const uint64_t pol_keep = ptx::createpolicy_evict_last(), pol_drop = ptx::createpolicy_evict_first();
     // one thread: copy the chunk of ring use j into its slot (the first read keeps its
@@ -914,18 +932,52 @@ __global__ void __launch_bounds__(PT_THREADS, 1) rq_persist_kernel(const PTParam
         }
         for (int64_t j = 0; j < min(2 * nb, (int64_t)PT_RING); ++j) issue(j);
     }
-    // ---- phase 1: a_max of the registers, the spill chunks and the held part
+    // ---- phase 1: a_max of the registers, the TMEM part, the spill chunks and the held part
     uint4 reg[PT_REG_VEC];
 #pragma unroll
     for (int j = 0; j < PT_REG_VEC; ++j) {
         const int64_t k = r0 + t + (int64_t)PT_THREADS * j;
-        reg[j] = k < v1 ? ld_v4_stream(xv + k) : make_uint4(0, 0, 0, 0);
+        reg[j] = k < r1 ? ld_v4_stream(xv + k) : make_uint4(0, 0, 0, 0);
     }
     uint32_t m2 = 0;
+    // the TMEM part, PT_TMEM_BATCH vectors at a time: batch i's loads go out one spill
+    // chunk before its max and its store, so that their latency overlaps the stream
+    constexpr int NTB = PT_TMEM_VEC / PT_TMEM_BATCH;
+    uint4 tb[PT_TMEM_BATCH];
+    int next_tb = 0;
+    auto load_tb = [&](int i) {
+#pragma unroll
+        for (int u = 0; u < PT_TMEM_BATCH; ++u) {
+            const int64_t k = r1 + t + (int64_t)PT_THREADS * (i * PT_TMEM_BATCH + u);
+            tb[u] = k < v1 ? ld_v4_stream(xv + k) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    auto store_tb = [&](int i) {                       // warp-collective
+        uint32_t w[16];
+#pragma unroll
+        for (int u = 0; u < PT_TMEM_BATCH; ++u) {
+            m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(tb[u]));
+            w[4 * u] = tb[u].x;
+            w[4 * u + 1] = tb[u].y;
+            w[4 * u + 2] = tb[u].z;
+            w[4 * u + 3] = tb[u].w;
+        }
+        ptx::tmem_st_32x32b_x16(tmem + (uint32_t)(16 * i), w);
+    };
+    load_tb(0);
     // phase 1's ring also sends out phase 2's first copies as the ring empties
     bool fail = !run_ring(0, nb, 2 * nb, [&](const uint4* sv, int64_t, int64_t nv) {
         for (int64_t k = t; k < nv; k += PT_THREADS) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(sv[k]));
+        if (next_tb < NTB) {
+            store_tb(next_tb);
+            if (++next_tb < NTB) load_tb(next_tb);
+        }
     });
+    while (next_tb < NTB) {
+        store_tb(next_tb);
+        if (++next_tb < NTB) load_tb(next_tb);
+    }
+    ptx::tmem_st_wait();
 #pragma unroll
     for (int j = 0; j < PT_REG_VEC; ++j) m2 = bmax_abs_bf16x2(m2, vec_amax2_bf(reg[j]));
     for (int c = 0; c < nhc; ++c) fail |= !pt_wait_copy(&hbar[c], 0, p.status);
@@ -969,6 +1021,9 @@ __global__ void __launch_bounds__(PT_THREADS, 1) rq_persist_kernel(const PTParam
         if (t == 0)
             for (int64_t j = nb; j < min(2 * nb, nb + (int64_t)PT_RING); ++j)
                 pt_wait_copy(&rbar[j % PT_RING], (uint32_t)((j / PT_RING) & 1), p.status);
+        ptx::tc_fence_before();
+        __syncthreads();                               // every thread's TMEM stores are complete
+        if (warp == 0) ptx::tmem_dealloc(s_tmem, PT_TMEM_COLS);
         return;
     }
     gm = block_max_u32(gm, red);
@@ -995,9 +1050,22 @@ __global__ void __launch_bounds__(PT_THREADS, 1) rq_persist_kernel(const PTParam
 #pragma unroll
     for (int j = 0; j < PT_REG_VEC; ++j) {
         const int64_t k = r0 + t + (int64_t)PT_THREADS * j;
-        if (k < v1) emit(k, reg[j]);
+        if (k < r1) emit(k, reg[j]);
+    }
+    for (int i = 0; i < NTB; ++i) {                    // warp-collective loads
+        uint32_t w[16];
+        ptx::tmem_ld_32x32b_x16(tmem + (uint32_t)(16 * i), w);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < PT_TMEM_BATCH; ++u) {
+            const int64_t k = r1 + t + (int64_t)PT_THREADS * (i * PT_TMEM_BATCH + u);
+            if (k < v1) emit(k, make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]));
+        }
     }
     for (int64_t k = t; k < n_held; k += PT_THREADS) emit(v0 + k, *reinterpret_cast<const uint4*>(held + k * 16));
+    ptx::tc_fence_before();
+    __syncthreads();                                   // every thread's TMEM loads are complete
+    if (warp == 0) ptx::tmem_dealloc(s_tmem, PT_TMEM_COLS);
 }
 
 // ================================================================ launchers
