@@ -65,3 +65,30 @@ def test_per_row_beyond_2pow31_elements(big_input):
     got = q.cpu().numpy()
     del q
     assert np.array_equal(got.reshape(-1), rq.reshape(-1))
+
+
+def test_gemm_output_beyond_2pow31_elements():
+    """Y [65536, 32768] (2^31 outputs, 4.3 GB of bf16) from the CTA-pair kernel with
+    per-row scales, K = 256; 8,192 sampled outputs, the last rows and columns among them,
+    against the oracle under the acceptance rule."""
+    M, N, K = 65536, 32768, 256
+    g = np.random.default_rng(91)
+    qa = g.integers(0, 0x7E, (M, K), dtype=np.uint8) | (g.integers(0, 2, (M, K), dtype=np.uint8) << 7)
+    qb = g.integers(0, 0x7E, (N, K), dtype=np.uint8) | (g.integers(0, 2, (N, K), dtype=np.uint8) << 7)
+    sa = np.exp(g.standard_normal(M)).astype(np.float32) * np.float32(1e-3)
+    sb = np.exp(g.standard_normal(N)).astype(np.float32) * np.float32(1e-3)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8.fp8_scaled_gemm(torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(), fp8.FP8_SCALE_ROW, fp8.FP8_E4M3,
+                        torch.from_numpy(qb).cuda(), torch.from_numpy(sb).cuda(), fp8.FP8_SCALE_ROW, fp8.FP8_E4M3,
+                        y, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    pm = np.concatenate([g.integers(0, M, 8000), np.full(96, M - 1), np.arange(M - 96, M)])
+    pn = np.concatenate([g.integers(0, N, 8000), np.arange(N - 96, N), np.full(96, N - 1)])
+    yv = y[torch.from_numpy(pm).cuda(), torch.from_numpy(pn).cuda()].float().cpu().numpy().astype(np.float64)
+    del y
+    torch.cuda.empty_cache()
+    y_ref, bound = oracle.gemm_ref_points(qa, sa, oracle.ROW, fp8.FP8_E4M3, qb, sb, oracle.ROW, fp8.FP8_E4M3, pm, pn)
+    ok, err, _ = oracle.gemm_within_tolerance(yv, y_ref, bound)
+    assert ok.all(), f"{int((~ok).sum())} sampled outputs off the oracle (max err {err.max():.3g})"
