@@ -85,6 +85,14 @@ def source_digest():
     return h.hexdigest()[:16]
 
 
+def use_sustained_peak(timed_ms: float, clocks: dict):
+    """The roofline denominator follows the run: the sustained (power-capped) FP8 figure
+    only when the timed region lasted at least 1 s and the sampled clocks saw the power
+    cap, else the burst figure.  Returns (use the sustained figure, power cap seen)."""
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    return timed_ms >= 1000.0 and capped, capped
+
+
 def profiled_traffic(kernel_tag: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel sources (the summary records the source digest)."""
@@ -902,10 +910,7 @@ def main():
     q_avg = statistics.mean(q_ms)
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP8_OVER_BF16
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_OVER_BF16
-    # the denominator follows the run: the sustained (power-capped) figure only when the
-    # timed region is long (>= 1 s) and the clocks saw the power cap, else the burst one
-    capped = "sw_power_cap" in (clocks.get("reasons") or [])
-    use_sustained = total_ms >= 1000.0 and capped
+    use_sustained, capped = use_sustained_peak(total_ms, clocks)
     fp8_peak = sustained if use_sustained else burst
     gemm_tflops = flops / (g_avg * 1e-3) / 1e12
     variant = {1: "ROWSCALE", 2: "BLOCK", 4: "MX"}[wl["x_mode"]]
